@@ -1,0 +1,165 @@
+"""fp64 CPU oracle for the TokenGate pruned-prefill hot path.
+
+TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the
+benchmark's CPU-baseline leg may import this package; the library never does,
+and it shares no code with the CUDA path.
+
+Two independent implementations live here:
+  * ``oracle.c`` -- plain C, fp64, OpenMP over output rows (``liboracle.so``,
+    compiled on first use or by ``oracle.build.build()``);
+  * ``twin``     -- the same definitions in numpy fp64, for small sizes only.
+
+Source: the MarkTechPost TokenGate article, sections "How does TokenGate
+learned token pruning work?" (gate, top-K, question never pruned, pruned
+forward) and "What is token-gated attention?" (score as logit bias, per-head
+gain, temperature).  Each function below restates the definition it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        vp, i64, i32, f64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        L.orc_gate_score.argtypes = [vp, i64, i32, vp, vp, vp, vp, i32, vp]
+        L.orc_gate_score.restype = None
+        L.orc_select_topk.argtypes = [vp, vp, i64, i64, vp]
+        L.orc_select_topk.restype = i64
+        L.orc_gather.argtypes = [vp, i32, vp, i64, vp, vp, vp]
+        L.orc_gather.restype = None
+        L.orc_gated_attention_rows.argtypes = [vp, vp, vp, vp, vp, f64, i64, i32, i32, i32, vp, i64, vp]
+        L.orc_gated_attention_rows.restype = None
+        L.orc_num_threads.argtypes = []
+        L.orc_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def num_threads() -> int:
+    return int(lib().orc_num_threads())
+
+
+def _bf16_bits(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype == torch.bfloat16
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _np(a, dtype) -> np.ndarray:
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------- gate
+def gate_score(hidden, W1, b1, W2, b2) -> np.ndarray:
+    """s_i = b2 + sum_j W2_j * SiLU(b1_j + W1[j,:] . x_i) in fp64 over the bf16 inputs."""
+    n, d = hidden.shape
+    h = W1.shape[0]
+    hb, w1, bb1, w2, bb2 = (_bf16_bits(t) for t in (hidden, W1, b1, W2, b2))
+    out = np.empty(n, dtype=np.float64)
+    lib().orc_gate_score(_ptr(hb), n, d, _ptr(w1), _ptr(bb1), _ptr(w2), _ptr(bb2), h, _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------- top-K
+def select_topk(scores, doc_mask, k: int) -> np.ndarray:
+    """Kept indices (ascending int32): the k best document tokens by (score desc, index asc),
+    NaN below everything, plus every question token."""
+    s = _np(scores, np.float32)
+    m = _np(doc_mask, np.uint8)
+    out = np.empty(max(len(s), 1), dtype=np.int32)
+    cnt = lib().orc_select_topk(_ptr(s), _ptr(m), len(s), int(k), _ptr(out))
+    return out[:cnt].copy()
+
+
+def select_topk_varlen(scores, doc_mask, cu_seqlens: Sequence[int], ks: Sequence[int]):
+    """Per-request selection of packed requests; indices are positions in the packed sequence.
+    Returns (kept_idx int32, cu_kept int32[B+1])."""
+    s = _np(scores, np.float32)
+    m = _np(doc_mask, np.uint8)
+    cu = [int(x) for x in cu_seqlens]
+    parts, cu_kept = [], [0]
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        kept = select_topk(s[lo:hi], m[lo:hi], int(ks[b])) + lo
+        parts.append(kept.astype(np.int32))
+        cu_kept.append(cu_kept[-1] + len(kept))
+    kept_all = np.concatenate(parts) if parts else np.zeros(0, np.int32)
+    return kept_all, np.asarray(cu_kept, dtype=np.int32)
+
+
+# --------------------------------------------------------------------------- gather
+def gather(hidden, kept, scores=None):
+    """hidden_k[r] = hidden[kept[r]] (bf16 bit patterns, uint16) and s_k[r] = scores[kept[r]]."""
+    hb = _bf16_bits(hidden)
+    n, d = hb.shape
+    kp = _np(kept, np.int32)
+    hk = np.empty((len(kp), d), dtype=np.uint16)
+    sk = None
+    sp = None
+    if scores is not None:
+        sp = _np(scores, np.float32)
+        sk = np.empty(len(kp), dtype=np.float32)
+    lib().orc_gather(_ptr(hb), d, _ptr(kp), len(kp), _ptr(hk),
+                     _ptr(sp) if sp is not None else None, _ptr(sk) if sk is not None else None)
+    return hk, sk
+
+
+# --------------------------------------------------------------------------- attention
+def gated_attention(Q, K, V, s, gain, tau: float, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """O[i,h] = sum_{j<=i} softmax_j(tau*Q_ih.K_jg/sqrt(D) + gain_h*s_j) V_jg, g = h // (Hq/Hkv).
+    Returns fp64 [len(rows), Hq, D] (all rows when ``rows`` is None)."""
+    S, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    qb, kb, vb = _bf16_bits(Q), _bf16_bits(K), _bf16_bits(V)
+    sv = _np(s, np.float32)
+    gv = _np(gain, np.float32)
+    r = np.arange(S, dtype=np.int64) if rows is None else _np(rows, np.int64)
+    out = np.empty((len(r), Hq, D), dtype=np.float64)
+    lib().orc_gated_attention_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(sv), _ptr(gv), float(tau),
+                                   S, Hq, Hkv, D, _ptr(r), len(r), _ptr(out))
+    return out
+
+
+def gated_attention_varlen(Q, K, V, s, gain, tau: float, cu_seqlens: Sequence[int],
+                           rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Packed requests: each segment [cu[b], cu[b+1]) attends causally within itself only.
+    ``rows`` are packed row indices (all rows when None); returns fp64 [len(rows), Hq, D]."""
+    cu = [int(x) for x in cu_seqlens]
+    S, Hq, D = Q.shape
+    rows_all = np.arange(S, dtype=np.int64) if rows is None else _np(rows, np.int64)
+    out = np.empty((len(rows_all), Hq, D), dtype=np.float64)
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        sel = np.nonzero((rows_all >= lo) & (rows_all < hi))[0]
+        if len(sel) == 0:
+            continue
+        out[sel] = gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], _np(s, np.float32)[lo:hi], gain, tau,
+                                   rows=rows_all[sel] - lo)
+    return out
+
+
+def sampled_rows(S: int, seed: int, head: int = 128, tail: int = 128, rand: int = 256) -> np.ndarray:
+    """Row sample for large cases: the first ``head`` rows, the last ``tail`` rows and ``rand``
+    seeded random rows in between (sorted, unique)."""
+    rng = np.random.default_rng(seed)
+    parts = [np.arange(min(head, S)), np.arange(max(0, S - tail), S)]
+    if S > head + tail:
+        parts.append(rng.choice(np.arange(head, S - tail), size=min(rand, S - head - tail), replace=False))
+    return np.unique(np.concatenate(parts)).astype(np.int64)

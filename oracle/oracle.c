@@ -1,0 +1,241 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for the TokenGate pruned-prefill hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load
+ * this file; only the tests, the package's smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header or table with the CUDA library.
+ *
+ * Source: the MarkTechPost article "Researchers from Stanford and UC Berkeley
+ * Introduce TokenGate: token-gated attention speeds up long-context prefill by up
+ * to 11.3x" (October 2026), called "the TokenGate article" below.  The article
+ * prints no formulas; where it is silent the plainest reading is taken and stated
+ * beside the function.
+ *
+ * Every floating-point computation runs in double precision over the exact
+ * values of the bf16 / fp32 inputs.  OpenMP parallelises only across independent
+ * output rows; the arithmetic of each row is a plain sequential loop in the
+ * order the definition is written.
+ *
+ * Parity pins (checked by tests/test_oracle_pins.py, independent of this file):
+ *   gate       -- torch.nn.functional linear+silu in fp64, the numpy twin,
+ *                 permutation / scaling / bias-shift invariants, W1 = 0 case.
+ *   select     -- O(n^2) rank counting brute force, hand-worked fixtures,
+ *                 |kept| = K + q, question always kept, ascending output.
+ *   gather     -- numpy fancy indexing.
+ *   attention  -- torch scaled_dot_product_attention in fp64 (GQA expanded,
+ *                 additive key bias), row 0 = V[0], bias-shift invariance,
+ *                 duplicated-KV-head equivalence, convex-hull bound,
+ *                 pruned keys never influence an output.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* bf16 -> double, exactly: a bf16 is the high half of an IEEE fp32. */
+static double bf16_value(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------ *
+ * Gate MLP scorer.
+ * TokenGate article, "How does TokenGate learned token pruning work?" (gate
+ * module): an MLP scores every token from its post-attention residual at gate
+ * layer L.  The article says only "small MLP"; the scorer taken here is
+ * Linear(d -> h), SiLU, Linear(h -> 1):
+ *     z_j = b1_j + sum_k W1[j,k] x_ik            (j < h)
+ *     a_j = z_j * sigmoid(z_j),  sigmoid(z) = 1 / (1 + exp(-z))
+ *     s_i = b2 + sum_j W2_j a_j
+ * No normalisation precedes the gate and the score is not squashed.
+ * hidden: bf16 [n, d] row-major; W1: bf16 [h, d] (row j = output unit j);
+ * b1, W2: bf16 [h]; b2: bf16 [1]; s: double [n].
+ * ------------------------------------------------------------------------ */
+void orc_gate_score(const uint16_t *hidden, int64_t n, int32_t d,
+                    const uint16_t *W1, const uint16_t *b1, const uint16_t *W2,
+                    const uint16_t *b2, int32_t h, double *s)
+{
+    double *w1 = (double *)malloc(sizeof(double) * (size_t)h * (size_t)d);
+    for (int64_t t = 0; t < (int64_t)h * d; ++t) w1[t] = bf16_value(W1[t]);
+    const double bias2 = bf16_value(b2[0]);
+
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(static)
+        for (int64_t i = 0; i < n; ++i) {
+            const uint16_t *row = hidden + (size_t)i * (size_t)d;
+            for (int32_t k = 0; k < d; ++k) x[k] = bf16_value(row[k]);
+            double out = 0.0;
+            for (int32_t j = 0; j < h; ++j) {
+                const double *wj = w1 + (size_t)j * (size_t)d;
+                double z = bf16_value(b1[j]);
+                for (int32_t k = 0; k < d; ++k) z += wj[k] * x[k];
+                const double a = z / (1.0 + exp(-z));
+                out += bf16_value(W2[j]) * a;
+            }
+            s[i] = out + bias2;
+        }
+        free(x);
+    }
+    free(w1);
+}
+
+/* ------------------------------------------------------------------------ *
+ * Top-K selection with the question always kept.
+ * TokenGate article, "How does TokenGate learned token pruning work?": a top-K
+ * selector keeps the highest-scoring tokens; only the document part of the
+ * prompt is prunable and the question is never pruned.
+ * Readings where the article is silent:
+ *   - ties go to the lower index; -0.0 and +0.0 compare equal (IEEE);
+ *   - NaN ranks below every number (below -inf), ties among NaNs by index;
+ *   - a budget above the document length keeps every document token.
+ * The order is a strict total order on (score, index), so the kept set is
+ * unique.  Output: kept indices in ascending order; returns their count.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    float s;
+    int32_t i;
+} scored_index;
+
+static int before(const scored_index *a, const scored_index *b)
+{
+    const int an = isnan(a->s), bn = isnan(b->s);
+    if (an != bn) return bn;               /* the non-NaN one comes first */
+    if (!an && a->s != b->s) return a->s > b->s;
+    return a->i < b->i;
+}
+
+static int cmp_rank(const void *pa, const void *pb)
+{
+    const scored_index *a = (const scored_index *)pa, *b = (const scored_index *)pb;
+    if (before(a, b)) return -1;
+    if (before(b, a)) return 1;
+    return 0;
+}
+
+int64_t orc_select_topk(const float *scores, const uint8_t *doc_mask, int64_t n,
+                        int64_t k, int32_t *kept)
+{
+    int64_t n_doc = 0;
+    for (int64_t i = 0; i < n; ++i) n_doc += doc_mask[i] != 0;
+    scored_index *doc = (scored_index *)malloc(sizeof(scored_index) * (size_t)(n_doc > 0 ? n_doc : 1));
+    int64_t t = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (doc_mask[i]) { doc[t].s = scores[i]; doc[t].i = (int32_t)i; ++t; }
+    qsort(doc, (size_t)n_doc, sizeof(scored_index), cmp_rank);
+
+    const int64_t take = k < 0 ? 0 : (k < n_doc ? k : n_doc);
+    uint8_t *keep = (uint8_t *)calloc((size_t)(n > 0 ? n : 1), 1);
+    for (int64_t r = 0; r < take; ++r) keep[doc[r].i] = 1;
+    for (int64_t i = 0; i < n; ++i)
+        if (!doc_mask[i]) keep[i] = 1;
+
+    int64_t m = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (keep[i]) kept[m++] = (int32_t)i;
+    free(keep);
+    free(doc);
+    return m;
+}
+
+/* ------------------------------------------------------------------------ *
+ * Gather / compaction.
+ * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
+ * forward): layers above L process only the kept tokens.
+ *     hidden_k[r, :] = hidden[kept[r], :],   s_k[r] = scores[kept[r]]
+ * ------------------------------------------------------------------------ */
+void orc_gather(const uint16_t *hidden, int32_t d, const int32_t *kept, int64_t n_kept,
+                uint16_t *hidden_k, const float *scores, float *s_k)
+{
+    for (int64_t r = 0; r < n_kept; ++r) {
+        memcpy(hidden_k + (size_t)r * (size_t)d, hidden + (size_t)kept[r] * (size_t)d,
+               sizeof(uint16_t) * (size_t)d);
+        if (scores && s_k) s_k[r] = scores[kept[r]];
+    }
+}
+
+/* ------------------------------------------------------------------------ *
+ * Token-gated causal GQA attention over the kept tokens.
+ * TokenGate article, "What is token-gated attention?": each kept token's score
+ * becomes a bias on the attention logits of the layers above the gate, with a
+ * learnable per-head gain and a learnable temperature.  The article prints no
+ * formula; the one taken here:
+ *     g      = h / (Hq / Hkv)                      (grouped KV head of q-head h)
+ *     l_ij   = tau * (Q[i,h,:] . K[j,g,:]) / sqrt(D) + gain_h * s_j,   j <= i
+ *     O[i,h] = sum_j softmax_j(l_i.) V[j,g,:]
+ * Causality is in compacted order, which is the original order because the
+ * kept indices are ascending.  Question keys carry their own score as bias.
+ * Q: bf16 [S, Hq, D]; K, V: bf16 [S, Hkv, D]; s: fp32 [S]; gain: fp32 [Hq].
+ * Only the rows listed in ``rows`` are computed (all rows for a full run);
+ * O: double [n_rows, Hq, D].
+ * ------------------------------------------------------------------------ */
+void orc_gated_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                              const float *s, const float *gain, double tau,
+                              int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                              const int64_t *rows, int64_t n_rows, double *O)
+{
+    const int32_t group = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    (void)S;
+
+#pragma omp parallel
+    {
+        double *q = NULL, *l = NULL;
+        int64_t l_cap = 0;
+        q = (double *)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n_rows * Hq; ++t) {
+            const int64_t r = t / Hq;
+            const int32_t hh = (int32_t)(t % Hq);
+            const int64_t i = rows[r];
+            const int32_t g = hh / group;
+            if (i + 1 > l_cap) {
+                free(l);
+                l_cap = i + 1;
+                l = (double *)malloc(sizeof(double) * (size_t)l_cap);
+            }
+            for (int32_t c = 0; c < D; ++c) q[c] = bf16_value(Q[((size_t)i * Hq + hh) * D + c]);
+            double m = -INFINITY;
+            for (int64_t j = 0; j <= i; ++j) {
+                const uint16_t *kj = K + ((size_t)j * Hkv + g) * D;
+                double dot = 0.0;
+                for (int32_t c = 0; c < D; ++c) dot += q[c] * bf16_value(kj[c]);
+                l[j] = tau * dot * inv_sqrt_d + (double)gain[hh] * (double)s[j];
+                if (l[j] > m) m = l[j];
+            }
+            double denom = 0.0;
+            double *o = O + ((size_t)r * Hq + hh) * D;
+            for (int32_t c = 0; c < D; ++c) o[c] = 0.0;
+            for (int64_t j = 0; j <= i; ++j) {
+                const double p = exp(l[j] - m);
+                denom += p;
+                const uint16_t *vj = V + ((size_t)j * Hkv + g) * D;
+                for (int32_t c = 0; c < D; ++c) o[c] += p * bf16_value(vj[c]);
+            }
+            for (int32_t c = 0; c < D; ++c) o[c] /= denom;
+        }
+        free(q);
+        free(l);
+    }
+}
+
+/* Number of OpenMP threads the oracle runs with (for reporting). */
+int orc_num_threads(void)
+{
+    int n = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            extern int omp_get_num_threads(void);
+            n = omp_get_num_threads();
+#endif
+        }
+    }
+    return n;
+}

@@ -1,0 +1,385 @@
+"""Pins of the fp64 CPU oracle against things other than itself.
+
+Each test ties an oracle function to a library routine (torch fp64), a brute
+force, a hand-worked example under tests/golden/, or an invariant the TokenGate
+article fixes (question never pruned, |kept| = K + question length, pruned keys
+never influence an output).  None of them retypes the oracle's own formula.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import twin
+from learned_token_pruning_mlp_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _rand_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(torch.bfloat16)
+
+
+# ============================================================================ gate
+def _gate_torch(hidden, W1, b1, W2, b2):
+    x = hidden.to(torch.float64)
+    z = F.linear(x, W1.to(torch.float64), b1.to(torch.float64))
+    return F.linear(F.silu(z), W2.to(torch.float64)[None, :], b2.to(torch.float64)).squeeze(-1).numpy()
+
+
+@pytest.mark.parametrize("n,d,h,seed", [(64, 32, 8, 0), (300, 256, 64, 1), (129, 72, 24, 2)])
+def test_gate_matches_torch_linear_silu(n, d, h, seed):
+    hidden = _rand_bf16((n, d), seed)
+    W1 = _rand_bf16((h, d), seed + 10, 1 / math.sqrt(d))
+    b1 = _rand_bf16((h,), seed + 11, 1 / math.sqrt(d))
+    W2 = _rand_bf16((h,), seed + 12, 1 / math.sqrt(h))
+    b2 = _rand_bf16((1,), seed + 13, 1 / math.sqrt(h))
+    ref = _gate_torch(hidden, W1, b1, W2, b2)
+    got = oracle.gate_score(hidden, W1, b1, W2, b2)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gate_matches_twin_on_tiny_workload():
+    w = W.get("tiny_n512")
+    args = W.gate_inputs(w)
+    np.testing.assert_allclose(oracle.gate_score(*args), twin.gate_score(*args), rtol=1e-12, atol=1e-12)
+
+
+def test_gate_zero_w1_gives_constant_library_value():
+    n, d, h = 17, 16, 8
+    hidden = _rand_bf16((n, d), 3)
+    W1 = torch.zeros((h, d), dtype=torch.bfloat16)
+    b1 = _rand_bf16((h,), 4)
+    W2 = _rand_bf16((h,), 5)
+    b2 = _rand_bf16((1,), 6)
+    expect = float((F.silu(b1.double()) * W2.double()).sum() + b2.double()[0])
+    got = oracle.gate_score(hidden, W1, b1, W2, b2)
+    np.testing.assert_allclose(got, np.full(n, expect), rtol=1e-13, atol=1e-13)
+
+
+def test_gate_invariances():
+    n, d, h = 40, 24, 12
+    hidden = _rand_bf16((n, d), 7)
+    W1 = _rand_bf16((h, d), 8, 0.3)
+    b1 = _rand_bf16((h,), 9)
+    W2 = _rand_bf16((h,), 10)
+    b2 = _rand_bf16((1,), 11)
+    base = oracle.gate_score(hidden, W1, b1, W2, b2)
+    # permuting the hidden units changes nothing
+    p = torch.randperm(h, generator=torch.Generator().manual_seed(0))
+    np.testing.assert_allclose(oracle.gate_score(hidden, W1[p], b1[p], W2[p], b2), base, rtol=1e-12, atol=1e-12)
+    # each token is scored from its own residual only
+    t = torch.randperm(n, generator=torch.Generator().manual_seed(1))
+    np.testing.assert_allclose(oracle.gate_score(hidden[t], W1, b1, W2, b2), base[t.numpy()], rtol=0, atol=0)
+    # b2 enters additively
+    b2s = (b2.float() + 2.0).to(torch.bfloat16)
+    delta = float(b2s[0]) - float(b2[0])
+    np.testing.assert_allclose(oracle.gate_score(hidden, W1, b1, W2, b2s) - delta, base, rtol=1e-12, atol=1e-12)
+    # the output layer is linear in W2
+    np.testing.assert_allclose(oracle.gate_score(hidden, W1, b1, W2 * 2, b2) - float(b2[0]),
+                               2 * (base - float(b2[0])), rtol=1e-12, atol=1e-12)
+
+
+def test_gate_one_hot_rows_reduce_to_elementwise_silu():
+    # W1 = identity (h = d), b1 = 0, W2 = e_j: the score is silu(x_j) + b2 (torch.nn.functional.silu)
+    d = 8
+    hidden = _rand_bf16((10, d), 12, 3.0)
+    W1 = torch.eye(d, dtype=torch.bfloat16)
+    b1 = torch.zeros(d, dtype=torch.bfloat16)
+    b2 = torch.zeros(1, dtype=torch.bfloat16)
+    for j in range(d):
+        W2 = torch.zeros(d, dtype=torch.bfloat16)
+        W2[j] = 1
+        got = oracle.gate_score(hidden, W1, b1, W2, b2)
+        np.testing.assert_allclose(got, F.silu(hidden[:, j].double()).numpy(), rtol=1e-14, atol=1e-300)
+
+
+# ============================================================================ top-K
+def _brute_topk(scores, mask, k):
+    """O(n^2) rank counting: document token i is kept iff fewer than k document tokens
+    precede it in (score desc with NaN last, index asc)."""
+    s = [float(x) for x in scores]
+    n = len(s)
+    keep = []
+    for i in range(n):
+        if not mask[i]:
+            keep.append(i)
+            continue
+        rank = 0
+        for j in range(n):
+            if j == i or not mask[j]:
+                continue
+            ni, nj = math.isnan(s[i]), math.isnan(s[j])
+            if ni and not nj:
+                rank += 1
+            elif ni == nj and not ni and s[j] > s[i]:
+                rank += 1
+            elif (ni == nj) and (ni or s[j] == s[i]) and j < i:
+                rank += 1
+        if rank < k:
+            keep.append(i)
+    return np.asarray(keep, dtype=np.int32)
+
+
+def _load_topk_golden():
+    with open(os.path.join(GOLDEN, "topk_worked.json")) as f:
+        g = json.load(f)
+    s = np.asarray([float(x) for x in g["scores"]], dtype=np.float32)
+    return g, s, np.asarray(g["doc_mask"], dtype=np.uint8)
+
+
+def test_topk_hand_worked_fixture():
+    g, s, m = _load_topk_golden()
+    for case in g["cases"]:
+        assert oracle.select_topk(s, m, case["k"]).tolist() == case["kept"], case
+        assert twin.select_topk(s, m, case["k"]).tolist() == case["kept"], case
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 48))
+    kind = seed % 4
+    if kind == 0:
+        s = rng.standard_normal(n).astype(np.float32)
+    elif kind == 1:
+        s = (rng.integers(0, 3, n) - 1).astype(np.float32)          # heavy ties
+    elif kind == 2:
+        s = rng.standard_normal(n).astype(np.float32)
+        s[rng.random(n) < 0.3] = np.nan
+        s[rng.random(n) < 0.2] = -0.0
+        s[rng.random(n) < 0.1] = -np.inf
+    else:
+        s = np.zeros(n, dtype=np.float32)                          # all equal
+    m = (rng.random(n) < 0.7).astype(np.uint8)
+    n_doc = int(m.sum())
+    for k in range(0, n_doc + 3):
+        ref = _brute_topk(s, m, k)
+        got = oracle.select_topk(s, m, k)
+        assert got.tolist() == ref.tolist(), (seed, k)
+        assert twin.select_topk(s, m, k).tolist() == ref.tolist(), (seed, k)
+
+
+def test_topk_invariants_on_mixture_scores():
+    n, q = 4096, 96
+    s = W.mixture_scores(n, seed=5).numpy()
+    m = np.ones(n, dtype=np.uint8)
+    m[-q:] = 0
+    for k in (0, 1, 100, 1000, n - q, n):
+        kept = oracle.select_topk(s, m, k)
+        kk = min(k, n - q)
+        assert len(kept) == kk + q                                   # |kept| = K + question length
+        assert set(range(n - q, n)) <= set(kept.tolist())            # question never pruned
+        assert np.all(np.diff(kept) > 0)                             # strictly ascending
+        doc_kept = np.asarray([i for i in kept if m[i]], dtype=np.int64)
+        pruned = np.setdiff1d(np.nonzero(m)[0], doc_kept)
+        if len(doc_kept) and len(pruned):
+            assert s[doc_kept].min() >= s[pruned].max()
+
+
+def test_topk_all_equal_keeps_lowest_indices():
+    n = 300
+    s = np.full(n, 1.5, dtype=np.float32)
+    m = np.ones(n, dtype=np.uint8)
+    m[::7] = 0
+    doc = np.nonzero(m)[0]
+    kept = oracle.select_topk(s, m, 50)
+    expect = np.union1d(doc[:50], np.nonzero(m == 0)[0])
+    assert kept.tolist() == expect.tolist()
+
+
+def test_topk_interleaved_question_tokens_kept():
+    rng = np.random.default_rng(3)
+    n = 200
+    s = rng.standard_normal(n).astype(np.float32)
+    m = (rng.random(n) < 0.5).astype(np.uint8)
+    for k in (0, 5, 50):
+        kept = oracle.select_topk(s, m, k)
+        assert set(np.nonzero(m == 0)[0].tolist()) <= set(kept.tolist())
+        assert kept.tolist() == _brute_topk(s, m, k).tolist()
+
+
+def test_topk_varlen_is_per_request():
+    cu = [0, 50, 50, 170, 171]
+    rng = np.random.default_rng(9)
+    n = cu[-1]
+    s = rng.standard_normal(n).astype(np.float32)
+    m = (rng.random(n) < 0.8).astype(np.uint8)
+    ks = [10, 3, 200, 0]
+    kept, cu_kept = oracle.select_topk_varlen(s, m, cu, ks)
+    for b in range(4):
+        lo, hi = cu[b], cu[b + 1]
+        seg = kept[cu_kept[b]:cu_kept[b + 1]]
+        assert seg.tolist() == (_brute_topk(s[lo:hi], m[lo:hi], ks[b]) + lo).tolist()
+
+
+# ============================================================================ gather
+def test_gather_matches_fancy_indexing():
+    hidden = _rand_bf16((100, 40), 21)
+    scores = torch.randn(100, generator=torch.Generator().manual_seed(2))
+    kept = np.asarray([0, 3, 4, 50, 99], dtype=np.int32)
+    hk, sk = oracle.gather(hidden, kept, scores)
+    assert np.array_equal(hk, hidden.view(torch.int16).numpy().view(np.uint16)[kept])
+    assert np.array_equal(sk, scores.numpy()[kept])
+
+
+# ============================================================================ attention
+def _sdpa_reference(Q, K, V, s, gain, tau):
+    """torch scaled_dot_product_attention in fp64 with GQA expanded and the gate score
+    as an additive float mask; causal handled through the mask."""
+    S, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    rep = Hq // Hkv
+    q = Q.double().permute(1, 0, 2)
+    k = K.double().repeat_interleave(rep, dim=1).permute(1, 0, 2)
+    v = V.double().repeat_interleave(rep, dim=1).permute(1, 0, 2)
+    causal = torch.ones(S, S, dtype=torch.bool).tril()
+    bias = gain.double()[:, None, None] * s.double()[None, None, :]
+    bias = bias.masked_fill(~causal[None], float("-inf"))
+    o = F.scaled_dot_product_attention(q, k, v, attn_mask=bias, scale=tau / math.sqrt(D))
+    return o.permute(1, 0, 2).numpy()
+
+
+def _attn_case(S, Hq, Hkv, D, seed):
+    Q = _rand_bf16((S, Hq, D), seed)
+    K = _rand_bf16((S, Hkv, D), seed + 1)
+    V = _rand_bf16((S, Hkv, D), seed + 2)
+    s = torch.randn(S, generator=torch.Generator().manual_seed(seed + 3))
+    gain = 0.5 + torch.rand(Hq, generator=torch.Generator().manual_seed(seed + 4))
+    return Q, K, V, s, gain
+
+
+def test_attention_plain_causal_when_gain_zero_tau_one():
+    # every document token kept, gain 0 and tau 1: ordinary causal attention
+    Q, K, V, s, _ = _attn_case(70, 4, 2, 32, 30)
+    gain = torch.zeros(4)
+    S, Hq, D = Q.shape
+    q = Q.double().permute(1, 0, 2)
+    k = K.double().repeat_interleave(2, dim=1).permute(1, 0, 2)
+    v = V.double().repeat_interleave(2, dim=1).permute(1, 0, 2)
+    ref = F.scaled_dot_product_attention(q, k, v, is_causal=True).permute(1, 0, 2).numpy()
+    got = oracle.gated_attention(Q, K, V, s, gain, 1.0)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("S,Hq,Hkv,D,tau", [(33, 4, 2, 16, 1.1), (64, 4, 4, 64, 0.7), (17, 8, 2, 8, 2.0)])
+def test_attention_matches_torch_sdpa_with_bias(S, Hq, Hkv, D, tau):
+    Q, K, V, s, gain = _attn_case(S, Hq, Hkv, D, 40 + S)
+    ref = _sdpa_reference(Q, K, V, s, gain, tau)
+    got = oracle.gated_attention(Q, K, V, s, gain, tau)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(twin.gated_attention(Q, K, V, s, gain, tau), got, rtol=1e-11, atol=1e-12)
+
+
+def test_attention_hand_worked_fixture():
+    with open(os.path.join(GOLDEN, "attention_worked.json")) as f:
+        g = json.load(f)
+    for ex in g["examples"]:
+        Q = _bf16(ex["Q"])[:, None, :]
+        K = _bf16(ex["K"])[:, None, :]
+        V = _bf16(ex["V"])[:, None, :]
+        s = np.asarray(ex["s"], dtype=np.float32)
+        gain = np.asarray([ex["gain"]], dtype=np.float32)
+        got = oracle.gated_attention(Q, K, V, s, gain, ex["tau"])[:, 0, :]
+        np.testing.assert_allclose(got, np.asarray(ex["O"]), rtol=0, atol=max(ex["tol"], 1e-15), err_msg=ex["name"])
+
+
+def test_attention_row_zero_is_v0_and_shift_invariance():
+    Q, K, V, s, gain = _attn_case(50, 4, 2, 32, 60)
+    o = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    rep = 2
+    for h in range(4):
+        assert np.array_equal(o[0, h], V[0, h // rep].double().numpy())
+    # adding the same constant to every key score leaves each softmax row unchanged
+    # (scores on a 2^-10 grid so that the fp32 shift is exact)
+    s = torch.round(s * 1024) / 1024
+    o = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    o2 = oracle.gated_attention(Q, K, V, s + 3.25, gain, 1.1)
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_temperature_scales_the_dot_product():
+    Q, K, V, s, gain = _attn_case(40, 4, 2, 16, 70)
+    a = oracle.gated_attention(Q, K, V, s, gain, 2.0)
+    b = oracle.gated_attention((Q.float() * 2).to(torch.bfloat16), K, V, s, gain, 1.0)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_gqa_equals_duplicated_kv_heads():
+    Q, K, V, s, gain = _attn_case(45, 8, 2, 16, 80)
+    a = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    b = oracle.gated_attention(Q, K.repeat_interleave(4, dim=1), V.repeat_interleave(4, dim=1), s, gain, 1.1)
+    np.testing.assert_allclose(a, b, rtol=0, atol=0)
+
+
+def test_attention_rows_inside_visible_value_hull():
+    Q, K, V, s, gain = _attn_case(64, 4, 2, 32, 90)
+    o = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    v = V.double().numpy()
+    for i in range(64):
+        for h in range(4):
+            vis = v[: i + 1, h // 2, :]
+            assert np.all(o[i, h] <= vis.max(axis=0) + 1e-12)
+            assert np.all(o[i, h] >= vis.min(axis=0) - 1e-12)
+
+
+def test_attention_sampled_rows_equal_full_rows():
+    Q, K, V, s, gain = _attn_case(300, 4, 2, 16, 95)
+    full = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    rows = oracle.sampled_rows(300, seed=1, head=10, tail=10, rand=20)
+    np.testing.assert_array_equal(oracle.gated_attention(Q, K, V, s, gain, 1.1, rows=rows), full[rows])
+
+
+def test_attention_varlen_is_block_diagonal():
+    Q, K, V, s, gain = _attn_case(90, 4, 2, 16, 97)
+    cu = [0, 30, 31, 90]
+    o = oracle.gated_attention_varlen(Q, K, V, s, gain, 1.1, cu)
+    for b in range(3):
+        lo, hi = cu[b], cu[b + 1]
+        np.testing.assert_array_equal(o[lo:hi], oracle.gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], s[lo:hi], gain, 1.1))
+
+
+# ============================================================================ pipeline
+def test_pruned_tokens_never_influence_outputs():
+    """Layers above the gate see only kept tokens and keep no KV for pruned ones: poisoning
+    every pruned position of the full-length inputs with NaN leaves the outputs bitwise equal
+    and NaN-free."""
+    w = W.get("tiny_n512")
+    hidden, W1, b1, W2, b2 = W.gate_inputs(w)
+    mask = W.doc_mask(w)
+    scores = oracle.gate_score(hidden, W1, b1, W2, b2).astype(np.float32)
+    kept = oracle.select_topk(scores, mask, 128)
+    assert len(kept) == 128 + 64
+    N = w.n
+    Qf, Kf, Vf = W.attention_inputs(w, N)
+    gain, tau = W.attention_params(w)
+    pruned = np.setdiff1d(np.arange(N), kept)
+
+    def run(Qf, Kf, Vf, sc, hid):
+        hk, sk = oracle.gather(hid, kept, sc)
+        o = oracle.gated_attention(Qf[kept], Kf[kept], Vf[kept], sk, gain, tau)
+        return hk, sk, o
+
+    clean = run(Qf, Kf, Vf, scores, hidden)
+    Qp, Kp, Vp, hp = Qf.clone(), Kf.clone(), Vf.clone(), hidden.clone()
+    sp = scores.copy()
+    nan = float("nan")
+    Qp[pruned] = nan
+    Kp[pruned] = nan
+    Vp[pruned] = nan
+    hp[pruned] = nan
+    sp[pruned] = nan
+    poisoned = run(Qp, Kp, Vp, sp, hp)
+    for a, b in zip(clean, poisoned):
+        assert np.array_equal(a, b)
+        assert not np.isnan(np.asarray(b, dtype=np.float64)).any()
