@@ -1,0 +1,417 @@
+"""Benchmark of the TokenGate pruned-prefill hot path on B200.
+
+One step = one pass of the whole path over one synthetic 128k-token request
+(hidden 2048, gate MLP 2048->256->1, question 512 tokens, budget K = 8192):
+    tg_gate_score (131072 tokens) -> tg_select_topk -> tg_gather (8704 rows)
+    -> 27 x tg_gated_attention (S = 8704, Hq 16, Hkv 8, D 128, independent Q/K/V per layer).
+
+Prints one JSON line.  ``value`` is the gated-attention algorithmic TFLOP/s of the
+whole step (27 layers of 4*D*Hq*S*(S+1)/2 flops divided by the full step time, the
+gate/top-K/gather time included); the gate+top-K+gather path is reported beside
+it in GB/s against HBM.  Inputs are resident in HBM before timing starts; the
+per-step working set (512 MiB residual + 1.9 GB of Q/K/V) is larger than L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {tokengate,reference}]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "qwen3_1p7b_n128k"
+METRIC = "gated-attn TFLOP/s & % bf16 peak; gate+topK+gather GB/s & % HBM, N=128k"
+DATASHEET_HBM_GBS = 8000.0
+
+
+def attention_flops(S: int, hq: int, d: int) -> int:
+    """Algorithmic flops of one causal gated-attention layer: QK^T and PV over the visible pairs."""
+    return 4 * d * hq * S * (S + 1) // 2
+
+
+def select_path_bytes(n: int, d: int, h: int, S: int) -> int:
+    """Algorithmic HBM bytes of gate + top-K + gather: each input read once, each output written once."""
+    gate = n * d * 2 + h * d * 2 + 3 * h * 2 + 2 + n * 4
+    topk = n * 4 + n * 1 + S * 4 + 4
+    gather = S * 4 + 2 * S * d * 2 + S * 4 + S * 4
+    return gate + topk + gather
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- tokengate arm
+def make_inputs(w, K):
+    from learned_token_pruning_mlp_b200 import workloads as W
+    hidden, W1, b1, W2, b2 = W.gate_inputs(w)
+    mask = W.doc_mask(w)
+    sel = W.selection_scores(w)
+    q = w.segments[0].q
+    S = K + q
+    gain, tau = W.attention_params(w)
+    layers = [W.attention_inputs(w, S, layer=l) for l in range(w.layers)]
+    return dict(hidden=hidden, W1=W1, b1=b1, W2=W2, b2=b2, mask=mask, sel=sel, gain=gain, tau=tau, layers=layers, S=S)
+
+
+def run_tokengate(args, world, rank, local):
+    import learned_token_pruning_mlp_b200 as tg
+    from learned_token_pruning_mlp_b200 import build as tgbuild
+    from learned_token_pruning_mlp_b200 import workloads as W
+    tgbuild.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.get(WORKLOAD)
+    K = args.budget
+    host = make_inputs(w, K)
+    S = host["S"]
+    n, d, h = w.n, w.d, w.h
+    L = w.layers
+
+    # device-resident copies
+    dv = {k: host[k].to(dev) for k in ("hidden", "W1", "b1", "W2", "b2", "mask", "sel", "gain")}
+    layers = [tuple(t.to(dev) for t in lay) for lay in host["layers"]]
+    scores = torch.empty(n, dtype=torch.float32, device=dev)
+    kept = torch.empty(n, dtype=torch.int32, device=dev)
+    n_kept = torch.empty(1, dtype=torch.int32, device=dev)
+    hidden_k = torch.empty(S, d, dtype=torch.bfloat16, device=dev)
+    s_k = torch.empty(S, dtype=torch.float32, device=dev)
+    outs = [torch.empty(S, w.hq, w.head_dim, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    stream = torch.cuda.current_stream(dev)
+    tau = host["tau"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tg.tg_gate_score(dv["hidden"], dv["W1"], dv["b1"], dv["W2"], dv["b2"], scores=scores)
+        tg.tg_select_topk(dv["sel"], dv["mask"], K, kept_idx=kept, n_kept=n_kept)
+        tg.tg_gather(dv["hidden"], kept, n_rows=S, n_kept=n_kept, hidden_k=hidden_k, scores=dv["sel"], s_k=s_k)
+        if ev is not None:
+            ev[1].record(stream)
+        for l in range(L):
+            Q, Kc, V = layers[l]
+            tg.tg_gated_attention(Q, Kc, V, s_k, dv["gain"], tau, O=outs[l])
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    bits = tg.tg_get_device_error()
+    if bits:
+        raise RuntimeError(f"device status bits {bits} after warm-up")
+    if int(n_kept.item()) != S:
+        raise RuntimeError(f"kept {int(n_kept.item())} tokens, expected {S}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    total_ms = start.elapsed_time(stop)
+    sel_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    att_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_per_step = max_over_ranks(total_ms / args.steps, world)
+    bits = tg.tg_get_device_error()
+    if bits:
+        raise RuntimeError(f"device status bits {bits} after timing")
+
+    flops_layer = attention_flops(S, w.hq, w.head_dim)
+    flops_step = flops_layer * L
+    sel_bytes = select_path_bytes(n, d, h, S)
+    peaks = load_peaks()
+    value = world * flops_step / (ms_per_step * 1e-3) / 1e12
+    att_launch_ms = statistics.mean(att_ms) / L
+    att_tflops = flops_layer / (att_launch_ms * 1e-3) / 1e12
+    sel_mean = statistics.mean(sel_ms)
+    sel_gbs = sel_bytes / (sel_mean * 1e-3) / 1e9
+
+    # end to end through the public calls with host buffers: H2D of the step's inputs
+    # from pinned memory and D2H of its results inside the timed region
+    e2e = run_e2e(tg, host, dev, w, K, S, tau, world, args)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: N=131072 (question 512), d=2048, gate 2048->256->1, K={K}, "
+                               f"S={S}, {L} gated layers Hq=16 Hkv=8 D=128",
+                   "global_batch": world, "seq_len": n, "kept": S, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (512 MiB residual + 1.9 GB Q/K/V per step)"},
+        "attention": {"ms_per_layer": round(att_launch_ms, 4), "tflops": round(att_tflops, 1),
+                      "frac_of_bf16_peak": round(att_tflops / peaks["bf16_tflops"], 4),
+                      "frac_of_bf16_sustained": round(att_tflops / peaks["bf16_tflops_sustained"], 4),
+                      "frac_of_nominal_2250": round(att_tflops / 2250.0, 4)},
+        "select_path": {"us": round(sel_mean * 1e3, 2), "bytes": sel_bytes, "gbs": round(sel_gbs, 1),
+                        "frac_of_hbm": round(sel_gbs / peaks["hbm_gbs"], 4),
+                        "frac_of_datasheet_8tbs": round(sel_gbs / DATASHEET_HBM_GBS, 4)},
+        "roofline": {"bound": "tensor", "achieved": round(att_tflops, 1), "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": round(att_tflops / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": None, "kernel": "gated_attention_kernel<128>",
+                     "peak_source": f"{peaks['source']} bf16 sustained (kernel timed inside a long step)"},
+        "e2e": e2e,
+        "gpu_launches": args.steps * (3 + L),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(host, w, S, budget_s=args.cpu_seconds)
+    return out
+
+
+def run_e2e(tg, host, dev, w, K, S, tau, world, args):
+    pin = lambda t: t.pin_memory()
+    h_in = {k: pin(host[k]) for k in ("hidden", "W1", "b1", "W2", "b2", "mask", "sel", "gain")}
+    h_layers = [tuple(pin(t) for t in lay) for lay in host["layers"]]
+    L = w.layers
+    d_in = {k: torch.empty_like(v, device=dev) for k, v in h_in.items()}
+    d_layers = [tuple(torch.empty_like(t, device=dev) for t in lay) for lay in h_layers]
+    scores = torch.empty(w.n, dtype=torch.float32, device=dev)
+    kept = torch.empty(w.n, dtype=torch.int32, device=dev)
+    n_kept = torch.empty(1, dtype=torch.int32, device=dev)
+    hidden_k = torch.empty(S, w.d, dtype=torch.bfloat16, device=dev)
+    s_k = torch.empty(S, dtype=torch.float32, device=dev)
+    outs = [torch.empty(S, w.hq, w.head_dim, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    h_kept = torch.empty(S, dtype=torch.int32).pin_memory()
+    h_outs = [torch.empty(S, w.hq, w.head_dim, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+    h2d = sum(v.numel() * v.element_size() for v in h_in.values()) + \
+        sum(t.numel() * t.element_size() for lay in h_layers for t in lay)
+    d2h = h_kept.numel() * 4 + sum(o.numel() * o.element_size() for o in h_outs)
+
+    def step():
+        for k in h_in:
+            d_in[k].copy_(h_in[k], non_blocking=True)
+        for l in range(L):
+            for a, b in zip(d_layers[l], h_layers[l]):
+                a.copy_(b, non_blocking=True)
+        tg.tg_gate_score(d_in["hidden"], d_in["W1"], d_in["b1"], d_in["W2"], d_in["b2"], scores=scores)
+        tg.tg_select_topk(d_in["sel"], d_in["mask"], K, kept_idx=kept, n_kept=n_kept)
+        tg.tg_gather(d_in["hidden"], kept, n_rows=S, n_kept=n_kept, hidden_k=hidden_k, scores=d_in["sel"], s_k=s_k)
+        for l in range(L):
+            Q, Kc, V = d_layers[l]
+            tg.tg_gated_attention(Q, Kc, V, s_k, d_in["gain"], tau, O=outs[l])
+            h_outs[l].copy_(outs[l], non_blocking=True)
+        h_kept.copy_(kept[:S], non_blocking=True)
+
+    steps = max(1, min(args.steps, 3))
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+    flops = attention_flops(S, w.hq, w.head_dim) * L
+    del d_in, d_layers, outs
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+def cpu_baseline(host, w, S, budget_s: float = 10.0, steps: int = 1):
+    """Time the fp64 CPU oracle on a bounded row sample of layer 0's attention; report TFLOP/s."""
+    import oracle
+    gain, tau = host["gain"], host["tau"]
+    Q, K, V = host["layers"][0]
+    s = torch.zeros(S)  # the key bias does not change the amount of work
+    # calibrate: rows near the end of the sequence cost ~S*4*D*Hq flops each
+    probe = np.arange(S - 4, S, dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.gated_attention(Q, K, V, s, gain, tau, rows=probe)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    per_row = dt / len(probe)
+    n_rows = int(max(4, min(S, budget_s / per_row)))
+    rows = np.arange(S - n_rows, S, dtype=np.int64)
+    flops = sum(4 * w.head_dim * w.hq * (int(r) + 1) for r in rows)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.gated_attention(Q, K, V, s, gain, tau, rows=rows)
+        times.append(time.perf_counter() - t0)
+    el = min(times)
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 C oracle, gated attention layer 0, last {n_rows} of {S} query rows x {w.hq} heads "
+                      f"(the longest causal rows), {flops:.3e} flops in {el:.2f} s"}
+
+
+def run_reference(args, world, rank):
+    """The slow oracle on the host cores, on the same workload (bounded sample per step)."""
+    if rank != 0:
+        return None
+    from learned_token_pruning_mlp_b200 import workloads as W
+    import oracle
+    w = W.get(WORKLOAD)
+    K = args.budget
+    q = w.segments[0].q
+    S = K + q
+    Q, Kc, V = W.attention_inputs(w, S, layer=0)
+    gain, tau = W.attention_params(w)
+    s = W.random_scores(S, 0)
+    n_rows = max(2, int(args.ref_rows))
+    rows = np.arange(S - n_rows, S, dtype=np.int64)
+    flops = sum(4 * w.head_dim * w.hq * (int(r) + 1) for r in rows)
+    for _ in range(args.warmup):
+        oracle.gated_attention(Q, Kc, V, s, gain, tau, rows=rows[:2])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gated_attention(Q, Kc, V, s, gain, tau, rows=rows)
+    el = (time.perf_counter() - t0) / args.steps
+    val = flops / el / 1e12
+    sample = (f"fp64 C oracle, gated attention layer 0 of {WORKLOAD} (S={S}), last {n_rows} query rows x "
+              f"{w.hq} heads per step ({flops:.3e} flops)")
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}: S={S} kept tokens, Hq=16 Hkv=8 D=128 (row sample)",
+                       "global_batch": 1, "seq_len": w.n, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
+    ap.add_argument("--budget", type=int, default=8192)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        out = run_tokengate(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

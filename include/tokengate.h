@@ -1,0 +1,202 @@
+/*
+ * tokengate.h -- C ABI of the B200 (sm_100a) TokenGate pruned-prefill library.
+ *
+ * The library implements the data-parallel core of the method described in the
+ * MarkTechPost article "Researchers from Stanford and UC Berkeley Introduce
+ * TokenGate: token-gated attention speeds up long-context prefill by up to
+ * 11.3x" (October 2026), called "the TokenGate article" below:
+ *
+ *   1. tg_gate_score      -- MLP gate scores every prompt token from its residual;
+ *   2. tg_select_topk     -- keep the K best document tokens, always keep the question;
+ *   3. tg_gather          -- compact the kept tokens' rows;
+ *   4. tg_gated_attention -- causal GQA attention over the kept tokens with the
+ *                            gate score as a per-key logit bias.
+ *
+ * Conventions shared by every call
+ *   - Tensor arguments are DEVICE pointers owned by the caller, packed row-major
+ *     (the last dimension contiguous).  The library never allocates, never
+ *     frees and never keeps a pointer after the call returns.
+ *   - bf16 tensors are passed as tg_bf16, the raw 16-bit pattern.
+ *   - Calls are asynchronous on ``stream`` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronise it.  They can be captured into a
+ *     CUDA graph.
+ *   - The return value reports errors that the host can detect (shapes,
+ *     alignment, null pointers, unsupported sizes, launch failures).  When it
+ *     is not TG_OK nothing was launched; tg_last_error_detail() describes it.
+ *   - Conditions only the device can see (an index out of range, a budget
+ *     above the document length, a full output, a bounded wait that ran out)
+ *     set bits in a sticky per-device status word and never trap.  Read and
+ *     clear it with tg_get_device_error().
+ *   - Calls on different streams may run concurrently; they share only the
+ *     status word, whose bits are OR-ed.
+ */
+#ifndef TOKENGATE_H
+#define TOKENGATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TG_ABI_VERSION 1
+
+typedef uint16_t tg_bf16;   /* bf16 bit pattern (the high half of an IEEE fp32) */
+typedef void *tg_stream;    /* cudaStream_t */
+
+typedef enum {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size */
+    TG_ERR_UNSUPPORTED = 2,   /* a size the kernels are not built for */
+    TG_ERR_ALIGNMENT = 3,     /* a pointer or row pitch not 16-byte aligned */
+    TG_ERR_CUDA = 4           /* a CUDA runtime/driver call failed (launch, attribute) */
+} tg_status;
+
+/* Bits of the per-device status word. */
+enum {
+    TG_DEVERR_TIMEOUT = 1u,    /* a bounded wait inside a kernel gave up; its outputs are invalid */
+    TG_DEVERR_INDEX_OOB = 2u,  /* tg_gather met an index outside [0, n); that row was skipped */
+    TG_DEVERR_K_GT_NDOC = 4u,  /* budget above the document length; clamped to keep every document token */
+    TG_DEVERR_CAPACITY = 8u,   /* kept tokens exceed the output capacity; writes past it were dropped */
+    TG_DEVERR_BAD_SEQLENS = 16u /* cu_seqlens not non-decreasing within [0, total] */
+};
+
+/* ABI version of the loaded library (TG_ABI_VERSION it was built with). */
+int tg_abi_version(void);
+
+/* Static string naming a status code. */
+const char *tg_status_string(tg_status status);
+
+/* Human-readable detail of the last non-TG_OK return on the calling host thread
+ * (empty string if none).  The pointer stays valid until that thread's next call. */
+const char *tg_last_error_detail(void);
+
+/* Synchronise ``stream``, then read and clear the status word of the current
+ * device into *bits (a host pointer).  Returns TG_ERR_CUDA if the
+ * synchronisation itself failed (e.g. a sticky CUDA error from another kernel). */
+tg_status tg_get_device_error(tg_stream stream, uint32_t *bits);
+
+/* Diagnostics: launch one kernel whose bounded wait on an mbarrier that nothing
+ * arrives on runs out after limit_ns (0 < limit_ns <= 2e9), so that the
+ * timeout path (TG_DEVERR_TIMEOUT in the status word) can be checked without
+ * hanging a GPU.  The paper has no counterpart; it exists for testing. */
+tg_status tg_probe_wait_timeout(int64_t limit_ns, tg_stream stream);
+
+/* --------------------------------------------------------------------------
+ * tg_gate_score -- gate MLP scorer.
+ * TokenGate article, "How does TokenGate learned token pruning work?" (gate
+ * module): a small MLP scores each token from its post-attention residual at
+ * the gate layer.  The scorer is Linear(d -> h), SiLU, Linear(h -> 1):
+ *     scores[i] = b2 + sum_j W2[j] * SiLU(b1[j] + sum_k W1[j,k] * hidden[i,k])
+ * computed with bf16 inputs, fp32 accumulation and an fp32 result.
+ *
+ *   hidden  bf16 [n, d]   residual stream at the gate layer
+ *   W1      bf16 [h, d]   first layer, nn.Linear layout (row j = hidden unit j)
+ *   b1      bf16 [h]
+ *   W2      bf16 [h]      second layer weights (one output)
+ *   b2      bf16 [1]
+ *   scores  fp32 [n]      output
+ * Sizes: n >= 0 (n = 0 launches nothing); d a positive multiple of 8;
+ * h a multiple of 16 in [16, 256].  hidden, W1 and scores 16-byte aligned.
+ * -------------------------------------------------------------------------- */
+tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d,
+                        const tg_bf16 *W1, const tg_bf16 *b1, const tg_bf16 *W2,
+                        const tg_bf16 *b2, int32_t h, float *scores, tg_stream stream);
+
+/* --------------------------------------------------------------------------
+ * tg_select_topk -- top-K over the document, question always kept.
+ * TokenGate article, "How does TokenGate learned token pruning work?": a top-K
+ * selector keeps the highest-scoring tokens; only the document part of the
+ * prompt is prunable, the question is never pruned.  The generation API's
+ * max_kept_prefill_tokens budget ("How do you deploy TokenGate?") is k.
+ *
+ * Among tokens with doc_mask[i] != 0 the k largest scores are kept, ordered by
+ * (score descending, index ascending): ties go to the lower index, -0.0 equals
+ * +0.0, NaN ranks below every number.  Every token with doc_mask[i] == 0 is
+ * kept.  kept_idx receives the union in ascending order and *n_kept (a device
+ * int32) its size, min(k, n_doc) + n_question.
+ *
+ *   scores    fp32 [n]      the gate scores (read only)
+ *   doc_mask  uint8 [n]     1 = document token (prunable), 0 = question token
+ *   k         budget, >= 0; k > n_doc keeps every document token and sets
+ *             TG_DEVERR_K_GT_NDOC
+ *   kept_idx  int32 [cap]   output; entries past *n_kept are left untouched
+ *   cap       capacity of kept_idx; writes past it are dropped and set
+ *             TG_DEVERR_CAPACITY
+ *   n_kept    int32 [1]     output (device)
+ * Sizes: 0 <= n < 2^31.  No workspace: intermediate state lives in the
+ * shared memory of one thread-block cluster.
+ * -------------------------------------------------------------------------- */
+tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask, int64_t n, int64_t k,
+                         int32_t *kept_idx, int64_t cap, int32_t *n_kept, tg_stream stream);
+
+/* Packed ragged batch: request b owns positions [cu_seqlens[b], cu_seqlens[b+1])
+ * of scores/doc_mask and budget k_per_seq[b] (both device int32 arrays).
+ * Kept indices are positions in the packed sequence; request b's come out at
+ * kept_idx[cu_kept[b] .. cu_kept[b+1]) and cu_kept (device int32 [B+1]) is
+ * written with cu_kept[0] = 0.  max_seqlen is a host upper bound on any
+ * request's length and total the packed length (the bound cu_seqlens must
+ * respect).  Malformed cu_seqlens set TG_DEVERR_BAD_SEQLENS. */
+tg_status tg_select_topk_varlen(const float *scores, const uint8_t *doc_mask,
+                                const int32_t *cu_seqlens, int32_t B, int64_t total,
+                                const int32_t *k_per_seq, int64_t max_seqlen,
+                                int32_t *kept_idx, int64_t cap, int32_t *cu_kept,
+                                tg_stream stream);
+
+/* --------------------------------------------------------------------------
+ * tg_gather -- compaction of the kept tokens.
+ * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
+ * forward): layers above the gate process only the kept tokens and create no
+ * KV entries for pruned ones.
+ *     hidden_k[r, :] = hidden[kept_idx[r], :]      s_k[r] = scores[kept_idx[r]]
+ * for r < n_rows, further limited to r < *n_kept when n_kept is not NULL (a
+ * device int32, e.g. the count written by tg_select_topk).  Rows outside
+ * that range are left untouched.
+ *
+ *   hidden    bf16 [n, d]      kept_idx  int32 [n_rows]   hidden_k bf16 [n_rows, d]
+ *   scores    fp32 [n] or NULL s_k       fp32 [n_rows] or NULL (both or neither)
+ * Sizes: d a positive multiple of 8, at most 16384; hidden and hidden_k
+ * 16-byte aligned.  An index outside [0, n) skips its row and sets TG_DEVERR_INDEX_OOB.
+ * -------------------------------------------------------------------------- */
+tg_status tg_gather(const tg_bf16 *hidden, int64_t n, int32_t d, const int32_t *kept_idx,
+                    int64_t n_rows, const int32_t *n_kept, tg_bf16 *hidden_k,
+                    const float *scores, float *s_k, tg_stream stream);
+
+/* --------------------------------------------------------------------------
+ * tg_gated_attention -- token-gated causal GQA attention over the kept tokens.
+ * TokenGate article, "What is token-gated attention?": each kept token's score
+ * becomes a bias on the attention logits of every layer above the gate, with a
+ * learnable per-head gain and a learnable temperature.  For query row i, query
+ * head h and key/value head g = h / (Hq / Hkv):
+ *     logit(i, j) = tau * (Q[i,h,:] . Kc[j,g,:]) / sqrt(D) + gain[h] * s[j],  j <= i
+ *     O[i,h,:]    = sum_j softmax_j(logit(i, .)) * V[j,g,:]
+ * Causality is in compacted order, which is the prompt order because kept
+ * indices are ascending.  bf16 inputs, fp32 accumulation, bf16 output.
+ *
+ *   Q   bf16 [S, Hq, D]    Kc, V  bf16 [S, Hkv, D]    O  bf16 [S, Hq, D]
+ *   s   fp32 [S]           gain   fp32 [Hq]           tau (host float)
+ * Sizes: S >= 0; D in {64, 128}; Hq a positive multiple of Hkv; S * Hq < 2^31.
+ * Q, Kc, V and O 16-byte aligned.
+ * -------------------------------------------------------------------------- */
+tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                             const float *s, const float *gain, float tau,
+                             int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                             tg_bf16 *O, tg_stream stream);
+
+/* Packed ragged batch: request b owns rows [cu_seqlens[b], cu_seqlens[b+1]) of
+ * Q, Kc, V, s and O (cu_seqlens: device int32 [B+1], e.g. cu_kept from
+ * tg_select_topk_varlen) and attends causally within itself only.  total is
+ * the packed row count and max_seqlen a host upper bound on any request's
+ * length (it sizes the grid). */
+tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                    const float *s, const float *gain, float tau,
+                                    const int32_t *cu_seqlens, int32_t B, int64_t total,
+                                    int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                    tg_bf16 *O, tg_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H */

@@ -1,1 +1,26 @@
-"""B200-native (sm_100a) library for the TokenGate pruned-prefill hot path."""
+"""B200-native (sm_100a) library for the TokenGate pruned-prefill hot path.
+
+The four calls (gate MLP scoring, top-K selection with the question kept, gather
+of the kept rows, token-gated causal GQA attention) run in hand-written CUDA
+kernels behind the C ABI of include/tokengate.h; this package is the thin
+ctypes binding over it (``_lib``) plus seeded synthetic workloads
+(``workloads``).  There is no CPU fallback.
+"""
+from ._lib import (  # noqa: F401
+    TG_DEVERR_BAD_SEQLENS,
+    TG_DEVERR_CAPACITY,
+    TG_DEVERR_INDEX_OOB,
+    TG_DEVERR_K_GT_NDOC,
+    TG_DEVERR_TIMEOUT,
+    TokenGateError,
+    lib,
+    tg_abi_version,
+    tg_gate_score,
+    tg_gated_attention,
+    tg_gated_attention_varlen,
+    tg_gather,
+    tg_get_device_error,
+    tg_probe_wait_timeout,
+    tg_select_topk,
+    tg_select_topk_varlen,
+)

@@ -1,0 +1,451 @@
+// attention.cu -- tg_gated_attention / tg_gated_attention_varlen: token-gated
+// causal GQA attention over the kept tokens.
+//
+// TokenGate article, "What is token-gated attention?": each kept token's gate
+// score becomes a bias on the attention logits of the layers above the gate,
+// with a learnable per-head gain and a learnable temperature.  For query row i,
+// head h, KV head g = h / (Hq/Hkv):
+//     logit(i,j) = tau * Q[i,h].K[j,g] / sqrt(D) + gain[h] * s[j]   (j <= i)
+//     O[i,h]     = softmax_j(logit(i,.)) V[., g]
+//
+// B200 design (flash-style, one CTA per pair of 128-row query tiles of one head):
+//   * TMEM (512 columns): S_0, S_1 (128 fp32 columns each, one per query tile),
+//     O_0, O_1 (D columns each).  The bf16 probabilities P_t are written back over
+//     the first 64 columns of S_t and fed to the PV product straight from TMEM.
+//   * warp 0 (one lane) loads Q once and streams K/V tiles of 128 keys through a
+//     TMA pipeline (128-byte swizzle); warp 3 copies the 128 key scores of each tile
+//     into shared memory with plain loads (request offsets need not be 16-byte
+//     aligned, which a TMA copy would require).
+//   * warp 1 (one lane) issues every tcgen05.mma: S_t = Q_t K_j^T (both operands
+//     K-major in shared memory) and O_t += P_t V_j (P from TMEM, V MN-major in shared
+//     memory).  The MMAs of one thread execute in issue order, so S_t(j+1) may be
+//     issued right after O_t += P_t(j) V_j even though it overwrites P_t(j).
+//   * warps 4-7 and 8-11 are the softmax warpgroups of tile 0 and tile 1 (one query
+//     row per thread).  Each reads its S row with tcgen05.ld, forms the base-2 logit
+//     with one FMA (scale * S + gain*log2e * s_j, the bias fused in), applies the
+//     causal mask on the diagonal tile, exponentiates, writes P and keeps the row sum.
+//     While one warpgroup works on its softmax the tensor core works on the other
+//     tile's products.
+//   * The running max is only moved when it grows by more than 2^8; then O_t is
+//     rescaled in TMEM (after S_t(j) completes, which orders after O_t's previous
+//     product).  Otherwise exponentials are taken against the stale max, which stays
+//     exact in fp32 and loses nothing in bf16.
+//   * The epilogue divides O by the row sum, converts to bf16 and stores the rows.
+//   * CTAs are ordered heaviest first (the longest causal rows), which the hardware
+//     block scheduler turns into a longest-processing-time schedule.
+#include <algorithm>
+#include <cmath>
+
+#include "ptx.cuh"
+#include "runtime.h"
+
+namespace {
+
+constexpr int kBM = 128;   // query rows per tile
+constexpr int kBN = 128;   // keys per KV tile
+constexpr int kThreads = 384;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-row x 64-column swizzled block (16 KB)
+
+template <int D>
+struct Cfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr uint32_t kTileBytes = kHalfBytes * kHalves;  // 128 rows x D bf16
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr uint32_t kBiasBytes = kBN * 4;
+  static constexpr size_t kSmem = 1024 + 2 * kTileBytes + 2 * static_cast<size_t>(kStages) * kTileBytes +
+                                  kStages * kBiasBytes + 256;
+};
+
+struct AttnCtl {
+  uint64_t q_full;
+  uint64_t k_full[4];
+  uint64_t v_full[4];
+  uint64_t kv_empty[4];
+  uint64_t bias_full[4];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_final;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    gated_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ key_scores,
+                           const float *__restrict__ gain, float scale_log2, const int32_t *__restrict__ cu_seqlens,
+                           int64_t S_single, int64_t total, int n_mblocks, int B, int Hq, int Hkv,
+                           __nv_bfloat16 *__restrict__ O, uint32_t *err) {
+  using C = Cfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem;                                  // [2][tile]
+  uint8_t *sK = sQ + 2 * C::kTileBytes;                // [NS][tile]
+  uint8_t *sV = sK + NS * C::kTileBytes;               // [NS][tile]
+  float *sBias = reinterpret_cast<float *>(sV + NS * C::kTileBytes);  // [NS][128] key scores
+  AttnCtl *ctl = reinterpret_cast<AttnCtl *>(reinterpret_cast<uint8_t *>(sBias) + NS * C::kBiasBytes);
+
+  // ---- work unit: heaviest query blocks first, then request, then head
+  const int per_mb = Hq * B;
+  const int mb = n_mblocks - 1 - static_cast<int>(blockIdx.x) / per_mb;
+  const int rest = static_cast<int>(blockIdx.x) % per_mb;
+  const int b = rest / Hq;
+  const int h = rest % Hq;
+  const int g = h / (Hq / Hkv);
+  int64_t seg_start = 0, len = S_single;
+  if (cu_seqlens) {
+    int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
+    s0 = s0 < 0 ? 0 : (s0 > total ? total : s0);
+    s1 = s1 < s0 ? s0 : (s1 > total ? total : s1);
+    seg_start = s0;
+    len = s1 - s0;
+  }
+  const int64_t row0 = static_cast<int64_t>(mb) * 2 * kBM;
+  if (row0 >= len) return;  // uniform over the CTA
+  const int n0 = 2 * mb + 1;                              // KV tiles of query tile 0 (its diagonal is tile 2mb)
+  const int n1 = (row0 + kBM < len) ? 2 * mb + 2 : 0;     // query tile 1 (0 = beyond the request)
+  const int n_kv = n1 ? n1 : n0;
+
+  const int warp = tg::warp_id();
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tg::mbar_init(tg::smem_addr(&ctl->q_full), 1);
+    for (int s = 0; s < NS; ++s) {
+      tg::mbar_init(tg::smem_addr(&ctl->k_full[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->v_full[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->kv_empty[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->bias_full[s]), 32);
+    }
+    for (int t = 0; t < 2; ++t) {
+      tg::mbar_init(tg::smem_addr(&ctl->s_full[t]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->p_full[t]), 128);
+    }
+    tg::mbar_init(tg::smem_addr(&ctl->o_final), 1);
+    tg::mbar_init(tg::smem_addr(&ctl->drain), 1);
+    ctl->abort_flag = 0;
+    tg::fence_mbar_init();
+    tg::prefetch_tmap(&tm_q);
+    tg::prefetch_tmap(&tm_k);
+    tg::prefetch_tmap(&tm_v);
+  }
+  if (warp == 2) {
+    tg::tmem_alloc(tg::smem_addr(&ctl->tmem_base), 512);
+    tg::tmem_relinquish();
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  tg::tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  volatile int *abort_flag = &ctl->abort_flag;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    const int nq = n1 ? 2 : 1;
+    const uint32_t qbar = tg::smem_addr(&ctl->q_full);
+    tg::mbar_arrive_expect_tx(qbar, nq * C::kTileBytes);
+    for (int t = 0; t < nq; ++t)
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tg::tma_load_3d(tg::smem_addr(sQ + t * C::kTileBytes + hf * kHalfBytes), &tm_q, qbar, hf * 64, h,
+                        static_cast<int32_t>(seg_start + row0 + t * kBM));
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j % NS;
+      const uint32_t ph = (j / NS) & 1;
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->kv_empty[s]), ph ^ 1u, abort_flag)) break;
+      const int32_t krow = static_cast<int32_t>(seg_start + static_cast<int64_t>(j) * kBN);
+      const uint32_t kb = tg::smem_addr(&ctl->k_full[s]);
+      tg::mbar_arrive_expect_tx(kb, C::kTileBytes);
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tg::tma_load_3d(tg::smem_addr(sK + s * C::kTileBytes + hf * kHalfBytes), &tm_k, kb, hf * 64, g, krow);
+      const uint32_t vb = tg::smem_addr(&ctl->v_full[s]);
+      tg::mbar_arrive_expect_tx(vb, C::kTileBytes);
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tg::tma_load_3d(tg::smem_addr(sV + s * C::kTileBytes + hf * kHalfBytes), &tm_v, vb, hf * 64, g, krow);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ key-score loader
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j % NS;
+      const uint32_t ph = (j / NS) & 1;
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->kv_empty[s]), ph ^ 1u, abort_flag)) break;
+#pragma unroll
+      for (int e = 0; e < kBN / 32; ++e) {
+        const int c = e * 32 + lane;
+        const int64_t kv = static_cast<int64_t>(j) * kBN + c;
+        sBias[s * kBN + c] = kv < len ? key_scores[seg_start + kv] : 0.f;
+      }
+      tg::mbar_arrive(tg::smem_addr(&ctl->bias_full[s]));
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
+    constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, D, false, true);
+    bool ok = tg::mbar_wait(tg::smem_addr(&ctl->q_full), 0, abort_flag);
+
+    auto issue_s = [&](int t, int j) {
+      const int s = j % NS;
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(t * kBN);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
+        const uint64_t ad = tg::smem_desc_sw128(tg::smem_addr(sQ + t * C::kTileBytes) + off, 16, 1024);
+        const uint64_t bd = tg::smem_desc_sw128(tg::smem_addr(sK + s * C::kTileBytes) + off, 16, 1024);
+        tg::mma_bf16_ss(d_tmem, ad, bd, idesc_s, kk > 0);
+      }
+      tg::mma_commit(tg::smem_addr(&ctl->s_full[t]));
+    };
+    auto issue_pv = [&](int t, int j) {
+      const int s = j % NS;
+      const uint32_t d_tmem = tmem_base + 256u + static_cast<uint32_t>(t * D);
+      const uint32_t p_tmem = tmem_base + static_cast<uint32_t>(t * kBN);
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        // 16 keys = 16 rows of V (2 swizzle groups of 8 rows, 2048 bytes); D blocks 16 KB apart
+        const uint64_t bd = tg::smem_desc_sw128(tg::smem_addr(sV + s * C::kTileBytes) + kk * 2048u, kHalfBytes, 1024);
+        tg::mma_bf16_ts(d_tmem, p_tmem + kk * 8u, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+    };
+    auto wait_k = [&](int j) {
+      return tg::mbar_wait(tg::smem_addr(&ctl->k_full[j % NS]), (j / NS) & 1u, abort_flag);
+    };
+
+    if (ok && (ok = wait_k(0))) {
+      tg::tc_fence_after();
+      issue_s(0, 0);
+      if (n1) issue_s(1, 0);
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int s = j % NS;
+      if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->v_full[s]), (j / NS) & 1u, abort_flag))) break;
+      bool next_k_ready = false;
+      if (j < n0) {
+        if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->p_full[0]), j & 1u, abort_flag))) break;
+        tg::tc_fence_after();
+        issue_pv(0, j);
+        if (j + 1 < n0) {
+          if (!(ok = wait_k(j + 1))) break;
+          next_k_ready = true;
+          tg::tc_fence_after();
+          issue_s(0, j + 1);
+        }
+      }
+      if (j < n1) {
+        if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->p_full[1]), j & 1u, abort_flag))) break;
+        tg::tc_fence_after();
+        issue_pv(1, j);
+        if (j + 1 < n1) {
+          if (!next_k_ready && !(ok = wait_k(j + 1))) break;
+          tg::tc_fence_after();
+          issue_s(1, j + 1);
+        }
+      }
+      tg::mma_commit(tg::smem_addr(&ctl->kv_empty[s]));
+    }
+    if (ok) tg::mma_commit(tg::smem_addr(&ctl->o_final));
+    if (*abort_flag) {
+      tg::mma_commit(tg::smem_addr(&ctl->drain));
+      int local_abort = 0;
+      tg::mbar_wait(tg::smem_addr(&ctl->drain), 0, &local_abort, 100000000ull);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
+    const int quarter = warp & 3;           // TMEM lane quarter
+    const int r = quarter * 32 + lane;      // row within the tile
+    const int n_t = t ? n1 : n0;
+    const int64_t rt = row0 + t * kBM;      // first row of the tile (request-relative)
+    const int diag = static_cast<int>(rt / kBN);
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_taddr = tmem_base + static_cast<uint32_t>(t * kBN) + lane_off;
+    const uint32_t o_taddr = tmem_base + 256u + static_cast<uint32_t>(t * D) + lane_off;
+    const float g2 = gain[h] * kLog2e;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_t; ++j) {
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->s_full[t]), j & 1u, abort_flag) ||
+          !tg::mbar_wait(tg::smem_addr(&ctl->bias_full[j % NS]), (j / NS) & 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tg::tc_fence_after();
+      uint32_t x[kBN];
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) tg::tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
+      tg::tmem_ld_wait();
+      const float4 *bias4 = reinterpret_cast<const float4 *>(sBias + (j % NS) * kBN);
+      const bool on_diag = (j == diag);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c4 = 0; c4 < kBN / 4; ++c4) {
+        const float4 bv = bias4[c4];
+        const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c4 * 4 + e;
+          float v = fmaf(__uint_as_float(x[c]), scale_log2, bb[e] * g2);
+          if (on_diag && c > r) v = -INFINITY;
+          x[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      if (m_new - m > kRescaleLog2) {
+        const float alpha = tg::ex2_approx(m - m_new);
+        l *= alpha;
+        if (j > 0) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tg::tmem_ld32(o_taddr + c * 32, o);
+            tg::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tg::tmem_st32(o_taddr + c * 32, o);
+          }
+        }
+        m = m_new;
+      }
+      float rowsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN / 2; ++c) {
+        const float p0 = tg::ex2_approx(__uint_as_float(x[2 * c]) - m);
+        const float p1 = tg::ex2_approx(__uint_as_float(x[2 * c + 1]) - m);
+        rowsum += p0 + p1;
+        x[c] = pack_bf16x2(p0, p1);  // in place: x[c] is no longer needed once read above
+      }
+      l += rowsum;
+      tg::tmem_st32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+      tg::tmem_st32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+      tg::tmem_st_wait();
+      tg::tc_fence_before();
+      tg::mbar_arrive(tg::smem_addr(&ctl->p_full[t]));
+    }
+    if (ok && n_t > 0 && tg::mbar_wait(tg::smem_addr(&ctl->o_final), 0, abort_flag)) {
+      tg::tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const int64_t row = rt + r;
+      __nv_bfloat16 *orow = O + ((seg_start + row) * Hq + h) * static_cast<int64_t>(D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tg::tmem_ld32(o_taddr + c * 32, o);
+        tg::tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (row < len) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+    }
+  }
+
+  tg::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && ctl->abort_flag) tg::set_device_error(err, TG_DEVERR_TIMEOUT);
+  if (warp == 2) {
+    tg::tc_fence_after();
+    tg::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int D>
+tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain, float tau,
+                 const int32_t *cu_seqlens, int32_t B, int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv,
+                 tg_bf16 *O, cudaStream_t stream, uint32_t *err) {
+  using C = Cfg<D>;
+  CUtensorMap tm_q, tm_k, tm_v;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(Hq), static_cast<uint64_t>(total)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hq) * D * 2};
+    const uint32_t box[3] = {64, 1, kBM};
+    if (!tg::encode_tmap(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return TG_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(Hkv), static_cast<uint64_t>(total)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hkv) * D * 2};
+    const uint32_t box[3] = {64, 1, kBN};
+    if (!tg::encode_tmap(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Kc, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return TG_ERR_CUDA;
+    if (!tg::encode_tmap(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return TG_ERR_CUDA;
+  }
+  static bool configured[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(gated_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(C::kSmem));
+    if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    configured[dev] = true;
+  }
+  const float scale_log2 = tau / std::sqrt(static_cast<float>(D)) * kLog2e;
+  const int n_mblocks = static_cast<int>((max_seqlen + 2 * kBM - 1) / (2 * kBM));
+  const int64_t grid = static_cast<int64_t>(n_mblocks) * Hq * B;
+  if (grid == 0) return TG_OK;
+  if (grid > 0x7FFFFFFFLL) return tg::fail(TG_ERR_UNSUPPORTED, "grid too large");
+  gated_attention_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(
+      tm_q, tm_k, tm_v, s, gain, scale_log2, cu_seqlens, cu_seqlens ? 0 : total, total, n_mblocks, B, Hq, Hkv,
+      reinterpret_cast<__nv_bfloat16 *>(O), err);
+  return tg::check_launch("gated_attention_kernel");
+}
+
+tg_status validate(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain,
+                   float tau, int64_t total, int32_t Hq, int32_t Hkv, int32_t D, tg_bf16 *O) {
+  if (total < 0) return tg::fail(TG_ERR_INVALID_ARG, "sequence length must be >= 0");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+    return tg::fail(TG_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv (got %d, %d)", Hq, Hkv);
+  if (D != 64 && D != 128) return tg::fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+  if (!std::isfinite(tau)) return tg::fail(TG_ERR_INVALID_ARG, "tau must be finite");
+  if (total * Hq >= 0x7FFFFFFFLL) return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
+  if (total == 0) return TG_OK;
+  if (!Q || !Kc || !V || !s || !gain || !O) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (!tg::aligned16(Q) || !tg::aligned16(Kc) || !tg::aligned16(V) || !tg::aligned16(O))
+    return tg::fail(TG_ERR_ALIGNMENT, "Q, Kc, V and O must be 16-byte aligned");
+  return TG_OK;
+}
+
+}  // namespace
+
+extern "C" tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
+                                        const float *gain, float tau, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                        tg_bf16 *O, tg_stream stream) {
+  tg::clear_detail();
+  tg_status st = validate(Q, Kc, V, s, gain, tau, S, Hq, Hkv, D, O);
+  if (st != TG_OK || S == 0) return st;
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, cs, err)
+                  : launch<64>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, cs, err);
+}
+
+extern "C" tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
+                                               const float *gain, float tau, const int32_t *cu_seqlens, int32_t B,
+                                               int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                               tg_bf16 *O, tg_stream stream) {
+  tg::clear_detail();
+  if (B < 0) return tg::fail(TG_ERR_INVALID_ARG, "B must be >= 0");
+  if (max_seqlen < 0 || max_seqlen > total) return tg::fail(TG_ERR_INVALID_ARG, "max_seqlen must be in [0, total]");
+  if (B > 0 && !cu_seqlens) return tg::fail(TG_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  tg_status st = validate(Q, Kc, V, s, gain, tau, total, Hq, Hkv, D, O);
+  if (st != TG_OK || total == 0 || B == 0) return st;
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, cs, err)
+                  : launch<64>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, cs, err);
+}

@@ -1,0 +1,37 @@
+// runtime.h -- host-side helpers shared by the TokenGate launchers: error detail,
+// the per-device status word, SM count and TMA tensor-map encoding.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tokengate.h"
+
+namespace tg {
+
+// Record a printf-style detail for tg_last_error_detail() and return ``st``.
+tg_status fail(tg_status st, const char *fmt, ...);
+
+// Clear the calling thread's detail (start of every API call).
+void clear_detail();
+
+// Device address of the current device's status word (the kernels OR bits into it).
+// Returns nullptr (and records a detail) if the address cannot be obtained.
+uint32_t *device_error_word();
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Map a pending CUDA error after a launch to TG_ERR_CUDA.
+tg_status check_launch(const char *what);
+
+// Encode a tiled TMA descriptor; strides_bytes has rank-1 entries (dimension 0 is dense).
+// Returns false (with a detail recorded) on failure.
+bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,
+                 const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                 CUtensorMapSwizzle swizzle);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace tg

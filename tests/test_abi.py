@@ -1,0 +1,111 @@
+"""Host-only checks of the C ABI: the library builds, loads, exports every call
+include/tokengate.h declares, and rejects bad arguments before any launch.
+No GPU is needed: every case here fails validation before the first CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learned_token_pruning_mlp_b200 import build as tgbuild
+from learned_token_pruning_mlp_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tokengate.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    tgbuild.build()
+    return _lib.lib()
+
+
+def test_header_declares_the_four_calls():
+    names = _declared()
+    for must in ("tg_gate_score", "tg_select_topk", "tg_gather", "tg_gated_attention",
+                 "tg_select_topk_varlen", "tg_gated_attention_varlen", "tg_get_device_error"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    missing = [n for n in _declared() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_symbol():
+    assert set(_declared()) <= set(_lib._SIGNATURES)
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.tg_abi_version() == 1
+    assert L.tg_status_string(0) == b"TG_OK"
+    assert L.tg_status_string(3) == b"TG_ERR_ALIGNMENT"
+    assert L.tg_status_string(99) == b"TG_ERR_UNKNOWN"
+
+
+def _detail(L):
+    return L.tg_last_error_detail().decode()
+
+
+def test_gate_rejects_bad_shapes(L):
+    assert L.tg_gate_score(None, 10, 7, None, None, None, None, 64, None, None) == 1          # d % 8
+    assert "multiple of 8" in _detail(L)
+    assert L.tg_gate_score(None, -1, 64, None, None, None, None, 64, None, None) == 1         # n < 0
+    assert L.tg_gate_score(None, 10, 64, None, None, None, None, 48 + 1, None, None) == 2     # h % 16
+    assert L.tg_gate_score(None, 10, 64, None, None, None, None, 512, None, None) == 2         # h > 256
+    assert L.tg_gate_score(None, 0, 64, None, None, None, None, 64, None, None) == 0          # n = 0: no-op
+    assert L.tg_gate_score(None, 10, 64, None, None, None, None, 64, None, None) == 1         # null pointers
+    p = ctypes.c_void_p(16 * 1000 + 2)                                                         # misaligned
+    assert L.tg_gate_score(p, 10, 64, p, p, p, p, 64, p, None) == 3
+
+
+def test_topk_rejects_bad_arguments(L):
+    one = ctypes.c_void_p(4096)
+    assert L.tg_select_topk(one, one, -1, 5, one, 10, one, None) == 1
+    assert L.tg_select_topk(one, one, 1 << 31, 5, one, 10, one, None) == 1
+    assert L.tg_select_topk(one, one, 10, -1, one, 10, one, None) == 1
+    assert L.tg_select_topk(one, one, 10, 5, one, 10, None, None) == 1
+    assert L.tg_select_topk(None, one, 10, 5, one, 10, one, None) == 1
+    assert L.tg_select_topk_varlen(one, one, one, -1, 10, one, 5, one, 10, one, None) == 1
+    assert L.tg_select_topk_varlen(one, one, one, 2, 10, one, 11, one, 10, one, None) == 1  # max_seqlen > total
+    assert L.tg_select_topk_varlen(one, one, None, 2, 10, one, 5, one, 10, one, None) == 1
+
+
+def test_gather_rejects_bad_arguments(L):
+    p = ctypes.c_void_p(4096)
+    assert L.tg_gather(p, 10, 12, p, 4, None, p, None, None, None) == 1                    # d % 8
+    assert L.tg_gather(p, 10, 32768, p, 4, None, p, None, None, None) == 2                 # d too large
+    assert L.tg_gather(p, 10, 16, p, 4, None, p, p, None, None) == 1                       # scores without s_k
+    assert L.tg_gather(p, 10, 16, p, 0, None, p, None, None, None) == 0                    # nothing to do
+    assert L.tg_gather(ctypes.c_void_p(4100), 10, 16, p, 4, None, p, None, None, None) == 3
+
+
+def test_attention_rejects_bad_arguments(L):
+    p = ctypes.c_void_p(4096)
+    f = ctypes.c_float(1.0)
+    assert L.tg_gated_attention(p, p, p, p, p, f, 10, 6, 4, 128, p, None) == 1             # Hq % Hkv
+    assert L.tg_gated_attention(p, p, p, p, p, f, 10, 4, 2, 96, p, None) == 2              # D
+    assert L.tg_gated_attention(p, p, p, p, p, ctypes.c_float(float("inf")), 10, 4, 2, 64, p, None) == 1
+    assert L.tg_gated_attention(p, p, p, p, p, f, 0, 4, 2, 64, p, None) == 0               # S = 0
+    assert L.tg_gated_attention(p, p, p, None, p, f, 10, 4, 2, 64, p, None) == 1
+    assert L.tg_gated_attention(ctypes.c_void_p(4104), p, p, p, p, f, 10, 4, 2, 64, p, None) == 3
+    assert L.tg_gated_attention_varlen(p, p, p, p, p, f, None, 2, 10, 5, 4, 2, 64, p, None) == 1
+    assert L.tg_gated_attention_varlen(p, p, p, p, p, f, p, 2, 10, 11, 4, 2, 64, p, None) == 1
+
+
+def test_probe_rejects_bad_limit(L):
+    assert L.tg_probe_wait_timeout(0, None) == 1
+    assert L.tg_probe_wait_timeout(3_000_000_000, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _lib.lib()
