@@ -26,7 +26,8 @@
 //     causal mask on the diagonal tile, exponentiates, writes P and keeps the row sum.
 //     While one warpgroup works on its softmax the tensor core works on the other
 //     tile's products.
-//   * The running max is only moved when it grows by more than 2^8; then O_t is
+//   * The running max is only moved when it grows by more than 2^8 for some row of
+//     the warp (decided per warp: TMEM access is warp-collective); then O_t is
 //     rescaled in TMEM (after S_t(j) completes, which orders after O_t's previous
 //     product).  Otherwise exponentials are taken against the stale max, which stays
 //     exact in fp32 and loses nothing in bf16.
@@ -271,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
-      if (!tg::mbar_wait(tg::smem_addr(&ctl->s_full[t]), j & 1u, abort_flag) ||
-          !tg::mbar_wait(tg::smem_addr(&ctl->bias_full[j % NS]), (j / NS) & 1u, abort_flag)) {
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->s_full[t]), j & 1u, abort_flag) ||
+          !tg::mbar_wait_warp(tg::smem_addr(&ctl->bias_full[j % NS]), (j / NS) & 1u, abort_flag)) {
         ok = false;
         break;
       }
@@ -298,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const float m_new = fmaxf(m, mx);
-      if (m_new - m > kRescaleLog2) {
+      // The decision is taken per warp: the TMEM loads and stores below are warp-collective.
+      if (__any_sync(0xFFFFFFFFu, m_new - m > kRescaleLog2)) {
         const float alpha = tg::ex2_approx(m - m_new);
         l *= alpha;
         if (j > 0) {
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::tc_fence_before();
       tg::mbar_arrive(tg::smem_addr(&ctl->p_full[t]));
     }
-    if (ok && n_t > 0 && tg::mbar_wait(tg::smem_addr(&ctl->o_final), 0, abort_flag)) {
+    if (ok && n_t > 0 && tg::mbar_wait_warp(tg::smem_addr(&ctl->o_final), 0, abort_flag)) {
       tg::tc_fence_after();
       const float inv_l = 1.0f / l;
       const int64_t row = rt + r;

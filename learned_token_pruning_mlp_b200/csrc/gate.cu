@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tc = 0;
     for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
       const uint32_t acc = tc & 1u, aph = (tc >> 1) & 1u;
-      if (!tg::mbar_wait(tg::smem_addr(&ctl->acc_full[acc]), aph, abort_flag)) break;
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->acc_full[acc]), aph, abort_flag)) break;
       tg::tc_fence_after();
       const uint32_t taddr = tmem_base + acc * static_cast<uint32_t>(h) + (static_cast<uint32_t>(quarter * 32) << 16);
       float sum = 0.f;

@@ -218,8 +218,12 @@ def test_attention_within_tolerance(S, Hq, Hkv, D):
 
 
 def test_attention_large_bias_and_temperature():
-    # strong biases force the running-max rescale path
+    # Strong biases force the running-max rescale path.  They also make rows nearly
+    # one-hot (O ~ one V row); V is halved so that |O| < 4, where bf16 output rounding
+    # (half an ulp, <= 2^-8 below 2) leaves room inside max-abs 1e-2 (above 4 the
+    # half-ulp alone is 2^-6 > 1e-2, for any bf16-output kernel).
     Q, K, V, s, gain = _attn_inputs(1536, 4, 2, 128, 77)
+    V = (V.float() * 0.5).to(torch.bfloat16)
     s = s * 12.0
     for tau in (0.25, 3.0):
         got = tg.tg_gated_attention(Q.to(DEV), K.to(DEV), V.to(DEV), s.to(DEV), gain.to(DEV), tau).float().cpu().numpy()
