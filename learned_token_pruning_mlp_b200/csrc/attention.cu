@@ -12,25 +12,31 @@
 //   * TMEM (512 columns): S_0, S_1 (128 fp32 columns each, one per query tile),
 //     O_0, O_1 (D columns each).  The bf16 probabilities P_t are written back over
 //     the first 64 columns of S_t and fed to the PV product straight from TMEM.
+//   * The key bias rides on the tensor core: with c_j = gain_h*log2(e)*s_j / scale
+//     (scale = tau*log2(e)/sqrt(D)), one extra K=16 MMA step multiplies a constant
+//     [1, 1, 0...] block of Q by a [hi(c_j), lo(c_j), 0...] block of K (c_j split
+//     into two bf16 parts, exact to 2^-16 relative), so S'_ij = q_i.k_j + c_j and the
+//     base-2 logit is scale * S'_ij: the softmax needs one FMA per logit, as without
+//     a bias.  tau < 0 negates the A operand (so the largest logit is still the
+//     largest S'); tau = 0 skips the Q.K steps.
 //   * warp 0 (one lane) loads Q once and streams K/V tiles of 128 keys through a
-//     TMA pipeline (128-byte swizzle); warp 3 copies the 128 key scores of each tile
-//     into shared memory with plain loads (request offsets need not be 16-byte
-//     aligned, which a TMA copy would require).
-//   * warp 1 (one lane) issues every tcgen05.mma: S_t = Q_t K_j^T (both operands
-//     K-major in shared memory) and O_t += P_t V_j (P from TMEM, V MN-major in shared
-//     memory).  The MMAs of one thread execute in issue order, so S_t(j+1) may be
-//     issued right after O_t += P_t(j) V_j even though it overwrites P_t(j).
+//     TMA pipeline (128-byte swizzle); warp 3 writes the c_j block of each tile into
+//     shared memory from plain loads of the scores (request offsets need not be
+//     16-byte aligned, which a TMA copy would require).
+//   * warp 1 (one lane) issues every tcgen05.mma: S_t = [1 Q] [c K]^T (K-major
+//     operands in shared memory) and O_t += P_t V_j (P from TMEM, V MN-major in
+//     shared memory).  The MMAs of one thread execute in issue order, so S_t(j+1) may
+//     be issued right after O_t += P_t(j) V_j even though it overwrites P_t(j).
 //   * warps 4-7 and 8-11 are the softmax warpgroups of tile 0 and tile 1 (one query
-//     row per thread).  Each reads its S row with tcgen05.ld, forms the base-2 logit
-//     with one FMA (scale * S + gain*log2e * s_j, the bias fused in), applies the
-//     causal mask on the diagonal tile, exponentiates, writes P and keeps the row sum.
-//     While one warpgroup works on its softmax the tensor core works on the other
-//     tile's products.
+//     row per thread): tcgen05.ld of the S' row, causal mask on the diagonal tile,
+//     8-way max, exp2 of one packed f32x2 FMA per pair, 8-way sum, bf16 pack,
+//     tcgen05.st of P.  While one warpgroup works on its softmax the tensor core
+//     works on the other tile's products.
 //   * The running max is only moved when it grows by more than 2^8 for some row of
 //     the warp (decided per warp: TMEM access is warp-collective); then O_t is
-//     rescaled in TMEM (after S_t(j) completes, which orders after O_t's previous
-//     product).  Otherwise exponentials are taken against the stale max, which stays
-//     exact in fp32 and loses nothing in bf16.
+//     rescaled in TMEM after P is stored (S_t(j) completing orders this after O_t's
+//     previous product).  Otherwise exponentials are taken against the stale max,
+//     which stays exact in fp32 and loses nothing in bf16.
 //   * The epilogue divides O by the row sum, converts to bf16 and stores the rows.
 //   * CTAs are ordered heaviest first (the longest causal rows), which the hardware
 //     block scheduler turns into a longest-processing-time schedule.
@@ -48,15 +54,17 @@ constexpr int kThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-row x 64-column swizzled block (16 KB)
+constexpr uint32_t kExtBytes = kBM * 16 * 2;   // one 128-row x 16-column unswizzled block (4 KB)
+constexpr uint32_t kExtLBO = kExtBytes / 2;    // columns 8..15 follow columns 0..7
+constexpr uint32_t kExtSBO = 128;              // 8 rows x 16 bytes per core matrix
 
 template <int D>
 struct Cfg {
   static constexpr int kHalves = D / 64;
   static constexpr uint32_t kTileBytes = kHalfBytes * kHalves;  // 128 rows x D bf16
   static constexpr int kStages = D == 128 ? 2 : 4;
-  static constexpr uint32_t kBiasBytes = kBN * 4;
   static constexpr size_t kSmem = 1024 + 2 * kTileBytes + 2 * static_cast<size_t>(kStages) * kTileBytes +
-                                  kStages * kBiasBytes + 256;
+                                  (1 + kStages) * static_cast<size_t>(kExtBytes) + 256;
 };
 
 struct AttnCtl {
@@ -92,8 +100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sQ = smem;                                  // [2][tile]
   uint8_t *sK = sQ + 2 * C::kTileBytes;                // [NS][tile]
   uint8_t *sV = sK + NS * C::kTileBytes;               // [NS][tile]
-  float *sBias = reinterpret_cast<float *>(sV + NS * C::kTileBytes);  // [NS][128] key scores
-  AttnCtl *ctl = reinterpret_cast<AttnCtl *>(reinterpret_cast<uint8_t *>(sBias) + NS * C::kBiasBytes);
+  uint8_t *sQx = sV + NS * C::kTileBytes;              // [128 x 16] block of ones (columns 0, 1)
+  uint8_t *sKx = sQx + kExtBytes;                      // [NS][128 x 16] blocks of c_j (columns 0, 1)
+  AttnCtl *ctl = reinterpret_cast<AttnCtl *>(sKx + NS * kExtBytes);
 
   // ---- work unit: heaviest query blocks first, then request, then head
   const int per_mb = Hq * B;
@@ -116,8 +125,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n1 = (row0 + kBM < len) ? 2 * mb + 2 : 0;     // query tile 1 (0 = beyond the request)
   const int n_kv = n1 ? n1 : n0;
 
+  // ---- logit scaling: base-2 logit = eff * S', S' = (+/-)(q.k + c_j)
+  const bool skip_qk = (scale_log2 == 0.f);
+  const float eff = skip_qk ? 1.f : fabsf(scale_log2);
+  const float cmul = gain[h] * kLog2e / (skip_qk ? 1.f : scale_log2);
+
   const int warp = tg::warp_id();
   const int lane = threadIdx.x & 31;
+
+  // constant [1, 1] columns of the extended Q block, zeros elsewhere (also in the c_j blocks)
+  for (uint32_t w = threadIdx.x; w < (1 + NS) * kExtBytes / 4; w += kThreads) {
+    uint32_t v = 0;
+    if (w < kExtLBO / 4 && (w & 3u) == 0) v = 0x3F803F80u;  // bf16 1.0 twice at the start of each row
+    reinterpret_cast<uint32_t *>(sQx)[w] = v;
+  }
+  tg::fence_proxy_async_smem();
 
   if (threadIdx.x == 0) {
     tg::mbar_init(tg::smem_addr(&ctl->q_full), 1);
@@ -173,34 +195,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         tg::tma_load_3d(tg::smem_addr(sV + s * C::kTileBytes + hf * kHalfBytes), &tm_v, vb, hf * 64, g, krow);
     }
   } else if (warp == 3) {
-    // ------------------------------------------------------------ key-score loader
+    // ------------------------------------------------------------ key-bias block writer
     for (int j = 0; j < n_kv; ++j) {
       const int s = j % NS;
       const uint32_t ph = (j / NS) & 1;
       if (!tg::mbar_wait(tg::smem_addr(&ctl->kv_empty[s]), ph ^ 1u, abort_flag)) break;
 #pragma unroll
       for (int e = 0; e < kBN / 32; ++e) {
-        const int c = e * 32 + lane;
-        const int64_t kv = static_cast<int64_t>(j) * kBN + c;
-        sBias[s * kBN + c] = kv < len ? key_scores[seg_start + kv] : 0.f;
+        const int r = e * 32 + lane;
+        const int64_t kv = static_cast<int64_t>(j) * kBN + r;
+        const float c = kv < len ? cmul * key_scores[seg_start + kv] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(c);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(c - __bfloat162float(hi));
+        const __nv_bfloat162 pr = __halves2bfloat162(hi, lo);
+        *reinterpret_cast<__nv_bfloat162 *>(sKx + s * kExtBytes + r * 16) = pr;  // row r, columns 0..1
       }
+      tg::fence_proxy_async_smem();
       tg::mbar_arrive(tg::smem_addr(&ctl->bias_full[s]));
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
+    const uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false) | (scale_log2 < 0.f ? (1u << 13) : 0u);
     constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, D, false, true);
     bool ok = tg::mbar_wait(tg::smem_addr(&ctl->q_full), 0, abort_flag);
 
     auto issue_s = [&](int t, int j) {
       const int s = j % NS;
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(t * kBN);
+      tg::mma_bf16_ss(d_tmem, tg::smem_desc_noswz(tg::smem_addr(sQx), kExtLBO, kExtSBO),
+                      tg::smem_desc_noswz(tg::smem_addr(sKx + s * kExtBytes), kExtLBO, kExtSBO), idesc_s, 0u);
+      if (!skip_qk) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
-        const uint64_t ad = tg::smem_desc_sw128(tg::smem_addr(sQ + t * C::kTileBytes) + off, 16, 1024);
-        const uint64_t bd = tg::smem_desc_sw128(tg::smem_addr(sK + s * C::kTileBytes) + off, 16, 1024);
-        tg::mma_bf16_ss(d_tmem, ad, bd, idesc_s, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
+          const uint64_t ad = tg::smem_desc_sw128(tg::smem_addr(sQ + t * C::kTileBytes) + off, 16, 1024);
+          const uint64_t bd = tg::smem_desc_sw128(tg::smem_addr(sK + s * C::kTileBytes) + off, 16, 1024);
+          tg::mma_bf16_ss(d_tmem, ad, bd, idesc_s, 1u);
+        }
       }
       tg::mma_commit(tg::smem_addr(&ctl->s_full[t]));
     };
@@ -216,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     auto wait_k = [&](int j) {
-      return tg::mbar_wait(tg::smem_addr(&ctl->k_full[j % NS]), (j / NS) & 1u, abort_flag);
+      return tg::mbar_wait(tg::smem_addr(&ctl->k_full[j % NS]), (j / NS) & 1u, abort_flag) &&
+             tg::mbar_wait(tg::smem_addr(&ctl->bias_full[j % NS]), (j / NS) & 1u, abort_flag);
     };
 
     if (ok && (ok = wait_k(0))) {
@@ -268,12 +300,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_taddr = tmem_base + static_cast<uint32_t>(t * kBN) + lane_off;
     const uint32_t o_taddr = tmem_base + 256u + static_cast<uint32_t>(t * D) + lane_off;
-    const float g2 = gain[h] * kLog2e;
-    float m = -INFINITY, l = 0.f;
+    const uint64_t eff2 = tg::f2_pack(eff, eff);
+    float m = -INFINITY, l = 0.f;           // running max of S' (S' units) and row sum
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
-      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->s_full[t]), j & 1u, abort_flag) ||
-          !tg::mbar_wait_warp(tg::smem_addr(&ctl->bias_full[j % NS]), (j / NS) & 1u, abort_flag)) {
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->s_full[t]), j & 1u, abort_flag)) {
         ok = false;
         break;
       }
@@ -282,51 +313,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c) tg::tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
       tg::tmem_ld_wait();
-      const float4 *bias4 = reinterpret_cast<const float4 *>(sBias + (j % NS) * kBN);
-      const bool on_diag = (j == diag);
-      float mx = -INFINITY;
+      if (j == diag) {
 #pragma unroll
-      for (int c4 = 0; c4 < kBN / 4; ++c4) {
-        const float4 bv = bias4[c4];
-        const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c4 * 4 + e;
-          float v = fmaf(__uint_as_float(x[c]), scale_log2, bb[e] * g2);
-          if (on_diag && c > r) v = -INFINITY;
-          x[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
+        for (int c = 0; c < kBN; ++c)
+          if (c > r) x[c] = __float_as_uint(-INFINITY);
       }
-      const float m_new = fmaxf(m, mx);
-      // The decision is taken per warp: the TMEM loads and stores below are warp-collective.
-      if (__any_sync(0xFFFFFFFFu, m_new - m > kRescaleLog2)) {
-        const float alpha = tg::ex2_approx(m - m_new);
-        l *= alpha;
-        if (j > 0) {
+      float mx[8];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tg::tmem_ld32(o_taddr + c * 32, o);
-            tg::tmem_ld_wait();
+      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(x[k]);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tg::tmem_st32(o_taddr + c * 32, o);
-          }
-        }
+      for (int c = 8; c < kBN; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = tg::fmax3(mx[k], __uint_as_float(x[c + k]), __uint_as_float(x[c + 8 + k]));
+      const float rmax = fmaxf(tg::fmax3(mx[0], mx[1], mx[2]), tg::fmax3(tg::fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+      const float m_new = fmaxf(m, rmax);
+      // taken per warp: the TMEM loads and stores of the rescale are warp-collective
+      const bool rescale = __any_sync(0xFFFFFFFFu, (m_new - m) * eff > kRescaleLog2);
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = tg::ex2_approx((m - m_new) * eff);
         m = m_new;
       }
-      float rowsum = 0.f;
+      const float nms = -m * eff;
+      const uint64_t nms2 = tg::f2_pack(nms, nms);
+      uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int c = 0; c < kBN / 2; ++c) {
-        const float p0 = tg::ex2_approx(__uint_as_float(x[2 * c]) - m);
-        const float p1 = tg::ex2_approx(__uint_as_float(x[2 * c + 1]) - m);
-        rowsum += p0 + p1;
+        const uint64_t arg = tg::f2_fma(tg::f2_pack(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), eff2, nms2);
+        float a0, a1;
+        tg::f2_unpack(arg, a0, a1);
+        const float p0 = tg::ex2_approx(a0), p1 = tg::ex2_approx(a1);
+        acc[c & 3] = tg::f2_add(acc[c & 3], tg::f2_pack(p0, p1));
         x[c] = pack_bf16x2(p0, p1);  // in place: x[c] is no longer needed once read above
       }
-      l += rowsum;
       tg::tmem_st32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
       tg::tmem_st32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+      float s0, s1, s2, s3, s4, s5, s6, s7;
+      tg::f2_unpack(acc[0], s0, s1);
+      tg::f2_unpack(acc[1], s2, s3);
+      tg::f2_unpack(acc[2], s4, s5);
+      tg::f2_unpack(acc[3], s6, s7);
+      l = fmaf(l, alpha, ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+      if (rescale && j > 0) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tg::tmem_ld32(o_taddr + c * 32, o);
+          tg::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tg::tmem_st32(o_taddr + c * 32, o);
+        }
+      }
       tg::tmem_st_wait();
       tg::tc_fence_before();
       tg::mbar_arrive(tg::smem_addr(&ctl->p_full[t]));

@@ -1,0 +1,94 @@
+"""Run one TokenGate call repeatedly on seeded inputs (for profilers and quick timing).
+
+    python -m learned_token_pruning_mlp_b200.runone attention --S 8704 --repeat 3
+    python -m learned_token_pruning_mlp_b200.runone gate --n 131072
+    python -m learned_token_pruning_mlp_b200.runone topk --n 131072 --k 8192
+    python -m learned_token_pruning_mlp_b200.runone gather --n 131072 --rows 8704
+
+Each call is timed with CUDA events on the launching stream (after one warm-up
+call) and the mean per-call time is printed.  Shapes default to the 128k-context
+Qwen3-1.7B-like workload (d 2048, h 256, Hq 16, Hkv 8, D 128).
+"""
+from __future__ import annotations
+
+import argparse
+import math
+
+import torch
+
+from . import _lib as tg
+from . import build as tgbuild
+from . import workloads as W
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("call", choices=["gate", "topk", "gather", "attention"])
+    ap.add_argument("--n", type=int, default=131072)
+    ap.add_argument("--d", type=int, default=2048)
+    ap.add_argument("--h", type=int, default=256)
+    ap.add_argument("--k", type=int, default=8192)
+    ap.add_argument("--rows", type=int, default=8704)
+    ap.add_argument("--S", type=int, default=8704)
+    ap.add_argument("--hq", type=int, default=16)
+    ap.add_argument("--hkv", type=int, default=8)
+    ap.add_argument("--D", type=int, default=128)
+    ap.add_argument("--tau", type=float, default=1.1)
+    ap.add_argument("--repeat", type=int, default=3)
+    a = ap.parse_args()
+    tgbuild.build()
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device="cpu").manual_seed(0)
+
+    if a.call == "gate":
+        hidden = torch.randn(a.n, a.d, generator=g).to(torch.bfloat16).to(dev)
+        W1 = (torch.randn(a.h, a.d, generator=g) / math.sqrt(a.d)).to(torch.bfloat16).to(dev)
+        b1 = torch.zeros(a.h, dtype=torch.bfloat16, device=dev)
+        W2 = (torch.randn(a.h, generator=g) / math.sqrt(a.h)).to(torch.bfloat16).to(dev)
+        b2 = torch.zeros(1, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(a.n, dtype=torch.float32, device=dev)
+        fn = lambda: tg.tg_gate_score(hidden, W1, b1, W2, b2, scores=out)
+    elif a.call == "topk":
+        s = W.mixture_scores(a.n, 3).to(dev)
+        m = torch.ones(a.n, dtype=torch.uint8, device=dev)
+        m[-512:] = 0
+        kept = torch.empty(a.n, dtype=torch.int32, device=dev)
+        nk = torch.empty(1, dtype=torch.int32, device=dev)
+        fn = lambda: tg.tg_select_topk(s, m, a.k, kept_idx=kept, n_kept=nk)
+    elif a.call == "gather":
+        hidden = torch.randn(a.n, a.d, generator=g).to(torch.bfloat16).to(dev)
+        sc = torch.randn(a.n, generator=g).to(dev)
+        idx = torch.sort(torch.randperm(a.n, generator=g)[:a.rows]).values.to(torch.int32).to(dev)
+        hk = torch.empty(a.rows, a.d, dtype=torch.bfloat16, device=dev)
+        sk = torch.empty(a.rows, dtype=torch.float32, device=dev)
+        fn = lambda: tg.tg_gather(hidden, idx, hidden_k=hk, scores=sc, s_k=sk)
+    else:
+        Q = torch.randn(a.S, a.hq, a.D, generator=g).to(torch.bfloat16).to(dev)
+        K = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
+        V = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
+        s = torch.randn(a.S, generator=g).to(dev)
+        gain = (0.5 + torch.rand(a.hq, generator=g)).to(dev)
+        O = torch.empty_like(Q)
+        fn = lambda: tg.tg_gated_attention(Q, K, V, s, gain, a.tau, O=O)
+
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.repeat):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.repeat
+    bits = tg.tg_get_device_error()
+    extra = ""
+    if a.call == "attention":
+        fl = 4 * a.D * a.hq * a.S * (a.S + 1) / 2
+        extra = f" {fl / ms / 1e9:.1f} TFLOP/s"
+    print(f"{a.call}: {ms * 1e3:.1f} us per call{extra} (status bits {bits})")
+    if bits:
+        raise SystemExit(1)
+
+
+if __name__ == "__main__":
+    main()

@@ -230,6 +230,22 @@ def test_attention_large_bias_and_temperature():
         assert_attn_close(got, oracle.gated_attention(Q, K, V, s, gain, tau))
 
 
+@pytest.mark.parametrize("tau", [-0.7, 0.0, 1e-3, 2.5])
+def test_attention_temperature_sign_and_zero(tau):
+    # tau < 0 flips the order of the logits (largest logit = smallest q.k), tau = 0 leaves
+    # only the key bias; both must follow the same definition
+    Q, K, V, s, gain = _attn_inputs(700, 4, 2, 128, 31)
+    got = tg.tg_gated_attention(Q.to(DEV), K.to(DEV), V.to(DEV), s.to(DEV), gain.to(DEV), tau).float().cpu().numpy()
+    assert_attn_close(got, oracle.gated_attention(Q, K, V, s, gain, tau))
+
+
+def test_attention_negative_gain():
+    Q, K, V, s, gain = _attn_inputs(513, 4, 2, 64, 32)
+    gain = gain - 1.2
+    got = tg.tg_gated_attention(Q.to(DEV), K.to(DEV), V.to(DEV), s.to(DEV), gain.to(DEV), 1.1).float().cpu().numpy()
+    assert_attn_close(got, oracle.gated_attention(Q, K, V, s, gain, 1.1))
+
+
 def test_attention_varlen():
     lens = [300, 1, 0, 1000, 129]
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
