@@ -7,14 +7,18 @@
 // the lower index, -0.0 == +0.0, NaN below every number.
 //
 // B200 design: the work is memory-trivial (5 bytes a token), so the cost is
-// latency.  One request is handled by one 8-CTA thread-block cluster; each CTA
-// owns a contiguous chunk of the request and keeps its 32-bit order keys in
-// shared memory.  Four 8-bit radix passes find the K-th largest key: every CTA
-// builds a shared-memory histogram, the cluster barrier publishes it and every
-// CTA sums the eight histograms through distributed shared memory, so all of
-// them agree on the digit without touching global memory.  The ordered
-// compaction then needs only two more cluster exchanges (tie counts and kept
-// counts per CTA) and block-wide prefix sums.  No workspace, no global atomics,
+// latency.  One request is handled by one 8-CTA thread-block cluster of 1024
+// threads each; every thread owns 16 consecutive positions (loaded with 16-byte
+// vector loads) and keeps their 32-bit order keys in registers (131072 positions per
+// cluster; longer requests re-derive the keys from the scores on every pass).  Up to
+// four 8-bit radix passes find the K-th largest key: each CTA builds a shared-memory
+// histogram of the remaining candidates, one cluster barrier publishes it, 256
+// threads sum the eight CTAs' histograms through distributed shared memory and one
+// warp scans the 256 totals, so every CTA agrees on the digit without touching
+// global memory.  A pass whose chosen bin holds exactly the keys still needed ends
+// the search early.  Histograms alternate between two buffers, so one barrier per
+// pass suffices.  The ordered compaction needs one scan of packed (tie, keep) counts
+// per CTA and one exchange of the per-CTA totals.  No workspace, no global atomics,
 // one launch for a single request.
 #include <cooperative_groups.h>
 
@@ -28,12 +32,11 @@ namespace cg = cooperative_groups;
 namespace {
 
 constexpr int kCluster = 8;
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kItems = 8;                   // consecutive positions per thread in a compaction tile
-constexpr int kTile = kThreads * kItems;    // 4096 positions per tile
-constexpr int kBins = 256;
-constexpr int kKeyCap = 16384;              // order keys cached per CTA (64 KB)
+constexpr int kItems = 16;                        // consecutive positions per thread
+constexpr int kRound = kThreads * kItems;         // positions per CTA per round (16384)
+constexpr int kBins = 256;                        // 8-bit digits, four passes at most
 
 // Order key: larger key = earlier in (score desc, NaN last).  0 marks a question
 // token (never competes), 1 is NaN, every number maps to >= 0x007FFFFF.
@@ -45,70 +48,64 @@ __device__ __forceinline__ uint32_t order_key(float f, bool doc) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-struct Scan {
-  int *warp_tot;  // [kWarps + 1]
+struct TopkShared {
+  uint32_t hist[2][kBins];     // double-buffered per-CTA histograms (read by the cluster)
+  uint32_t tot[kBins];         // cluster totals of the current pass
+  uint32_t wsum[kWarps + 1];
+  uint32_t sel_digit, sel_above, sel_count;
+  long long exch[2];           // ties (key == T) and certain keeps of this CTA: read by the cluster
+  long long bcast[2];          // tie_base, out_base
 };
 
-// Block-wide exclusive prefix sum of one int per thread (thread order = index order).
-// Returns the exclusive prefix; *total receives the block sum.  Contains barriers.
-__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
+// Block-wide exclusive prefix sum of one value per thread (thread order = index order).
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, TopkShared &sh, uint32_t *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+  uint32_t incl = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
     if (lane >= off) incl += t;
   }
-  if (lane == 31) warp_tot[warp] = incl;
+  if (lane == 31) sh.wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < kWarps ? warp_tot[lane] : 0;
-    int wi = w;
+    const uint32_t w = sh.wsum[lane];
+    uint32_t wi = w;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, wi, off);
+      const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, wi, off);
       if (lane >= off) wi += t;
     }
-    if (lane < kWarps) warp_tot[lane] = wi - w;  // exclusive warp offsets
-    if (lane == kWarps - 1) warp_tot[kWarps] = wi;
+    sh.wsum[lane] = wi - w;
+    if (lane == 31) sh.wsum[kWarps] = wi;
   }
   __syncthreads();
-  const int res = warp_tot[warp] + incl - v;
-  *total = warp_tot[kWarps];
-  __syncthreads();
+  const uint32_t res = sh.wsum[warp] + incl - v;
+  *total = sh.wsum[kWarps];
   return res;
 }
 
-struct TopkShared {
-  uint32_t hist[kBins];
-  uint32_t tot[kBins];
-  int warp_tot[kWarps + 1];
-  uint32_t sel_digit;
-  uint32_t sel_above;
-  long long exch[2];          // values other CTAs of the cluster read: [0] ties, [1] kept
-  long long red[kWarps];
-};
-
-__device__ __forceinline__ void cluster_sum_hist(cg::cluster_group &cluster, TopkShared &sh) {
+// Sum the eight CTAs' histograms of buffer ``buf`` (one bin per thread of the first 256),
+// then let warp 0 find the digit of the remaining-th largest candidate, scanning bins
+// from 255 down.  Publishes sel_digit, sel_above (candidates in higher bins) and
+// sel_count (candidates in the chosen bin); sel_digit = 256 if none qualifies.
+__device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster, TopkShared &sh, int buf,
+                                                     uint32_t remaining) {
   if (threadIdx.x < kBins) {
-    uint32_t s = 0;
+    uint32_t c = 0;
 #pragma unroll
-    for (int c = 0; c < kCluster; ++c) s += cluster.map_shared_rank(sh.hist, c)[threadIdx.x];
-    sh.tot[threadIdx.x] = s;
+    for (int r = 0; r < kCluster; ++r) c += cluster.map_shared_rank(&sh.hist[buf][0], r)[threadIdx.x];
+    sh.tot[threadIdx.x] = c;
   }
   __syncthreads();
-}
-
-// Pick the digit D of the remaining-th largest candidate from sh.tot (bins scanned from 255 down).
-__device__ __forceinline__ void select_digit(TopkShared &sh, uint32_t remaining) {
-  if ((threadIdx.x >> 5) == 0) {
-    const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     uint32_t c[8];
     uint32_t sum = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      c[j] = sh.tot[255 - 8 * lane - j];
-      sum += c[j];
+    for (int e = 0; e < 8; ++e) {
+      c[e] = sh.tot[kBins - 1 - 8 * lane - e];
+      sum += c[e];
     }
     uint32_t incl = sum;
 #pragma unroll
@@ -117,45 +114,40 @@ __device__ __forceinline__ void select_digit(TopkShared &sh, uint32_t remaining)
       if (lane >= off) incl += t;
     }
     const uint32_t excl = incl - sum;
-    if (excl < remaining && remaining <= incl) {
+    if (lane == 31) {
+      sh.wsum[kWarps] = incl;  // total candidates
+      sh.sel_digit = kBins;
+    }
+    __syncwarp();
+    if (remaining > 0 && excl < remaining && remaining <= incl) {
       uint32_t run = excl;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (run + c[j] >= remaining) {
-          sh.sel_digit = 255u - 8u * lane - j;
+      for (int e = 0; e < 8; ++e) {
+        if (run + c[e] >= remaining) {
+          sh.sel_digit = kBins - 1 - 8 * lane - e;
           sh.sel_above = run;
+          sh.sel_count = c[e];
           break;
         }
-        run += c[j];
+        run += c[e];
       }
     }
   }
   __syncthreads();
 }
 
-__device__ __forceinline__ long long block_sum_ll(long long v, TopkShared &sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xFFFFFFFFu, v, off);
-  if (lane == 0) sh.red[warp] = v;
-  __syncthreads();
-  long long s = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) s += sh.red[w];
-  __syncthreads();
-  return s;
-}
-
 // One cluster per request.  Single-request mode: cu_seqlens == nullptr, the request is
 // [0, n_single) with budget k_single, base 0, and the CTA of rank 0 writes *n_kept.
 // Varlen mode: request b = cluster index, range from cu_seqlens, budget k_per_seq[b],
 // output offset cu_kept[b] (computed beforehand by seg_offsets_kernel).
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
+// kResident: every CTA's chunk fits one round (<= 16384 positions), keys stay in
+// registers; otherwise the keys are re-derived from the scores on every pass.
+template <bool kResident>
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     topk_cluster_kernel(const float *__restrict__ scores, const uint8_t *__restrict__ mask, int64_t n_single,
                         int64_t k_single, const int32_t *__restrict__ cu_seqlens, const int32_t *__restrict__ k_per_seq,
                         const int32_t *__restrict__ cu_kept, int64_t total, int32_t *__restrict__ kept_idx,
-                        int64_t cap, int32_t *__restrict__ n_kept, int use_cache, uint32_t *err) {
-  extern __shared__ __align__(16) uint32_t keys[];
+                        int64_t cap, int32_t *__restrict__ n_kept, uint32_t *err) {
   __shared__ TopkShared sh;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -172,154 +164,192 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
   }
   if (k < 0) k = 0;
   const int64_t len = end - start;
-  const int64_t chunk = (len + kCluster - 1) / kCluster;
+  // chunk: a multiple of kItems so that a thread's positions never straddle two CTAs
+  const int64_t chunk = ((len + kCluster - 1) / kCluster + kItems - 1) / kItems * kItems;
   const int64_t lo = start + chunk * rank;
-  const int64_t hi = std::min<int64_t>(lo + chunk, end);
+  const int64_t hi = lo + chunk < end ? lo + chunk : end;
   const int m = lo < hi ? static_cast<int>(hi - lo) : 0;
-  // The launcher sizes the key cache from its length bound; a request longer than
-  // that bound falls back to reading the scores again on every pass.
-  if (chunk > kKeyCap) use_cache = 0;
+  const int rounds = kResident ? 1 : (m + kRound - 1) / kRound;
 
-  auto key_at = [&](int i) -> uint32_t {
-    if (use_cache) return keys[i];
-    return order_key(scores[lo + i], mask[lo + i] != 0);
+  // 16-byte vector loads when this CTA's chunk starts aligned (always for a single request
+  // with aligned buffers; varlen requests may start anywhere and then use scalar loads)
+  const bool vec = ((reinterpret_cast<uintptr_t>(scores + lo) | reinterpret_cast<uintptr_t>(mask + lo)) & 15u) == 0;
+  uint32_t keys[kItems];
+  // positions past the chunk get key 0 and are excluded from every count by valid()
+  auto load_keys = [&](int round) {
+    const int i0 = round * kRound + threadIdx.x * kItems;
+    if (vec && i0 + kItems <= m) {
+      float f[kItems];
+      const float4 *s4 = reinterpret_cast<const float4 *>(scores + lo + i0);
+#pragma unroll
+      for (int q = 0; q < kItems / 4; ++q) {
+        const float4 v = __ldg(s4 + q);
+        f[4 * q] = v.x;
+        f[4 * q + 1] = v.y;
+        f[4 * q + 2] = v.z;
+        f[4 * q + 3] = v.w;
+      }
+      const uint4 mv = __ldg(reinterpret_cast<const uint4 *>(mask + lo + i0));
+      const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+      for (int e = 0; e < kItems; ++e) keys[e] = order_key(f[e], ((mw[e >> 2] >> (8 * (e & 3))) & 0xFFu) != 0);
+    } else {
+#pragma unroll
+      for (int e = 0; e < kItems; ++e) {
+        const int i = i0 + e;
+        keys[e] = i < m ? order_key(scores[lo + i], mask[lo + i] != 0) : 0u;
+      }
+    }
   };
+  auto valid = [&](int round, int e) { return round * kRound + static_cast<int>(threadIdx.x) * kItems + e < m; };
 
-  // ---- pass 0: order keys, histogram of the top byte, document count
-  for (int b = threadIdx.x; b < kBins; b += kThreads) sh.hist[b] = 0;
+  if (kResident) load_keys(0);
+  if (threadIdx.x < 2 * kBins) (&sh.hist[0][0])[threadIdx.x] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < m; i += kThreads) {
-    const uint32_t key = order_key(scores[lo + i], mask[lo + i] != 0);
-    if (use_cache) keys[i] = key;
-    if (key) atomicAdd(&sh.hist[key >> 24], 1u);
-  }
-  __syncthreads();
-  cluster.sync();
-  cluster_sum_hist(cluster, sh);
+
+  // ---- radix passes over 8-bit digits, most significant first.  Pass p histograms the
+  // candidates (document keys whose higher digits equal the prefix found so far).
+  uint32_t prefix = 0, pmask = 0;
+  uint32_t remaining = static_cast<uint32_t>(k < 0x7FFFFFFFLL ? k : 0x7FFFFFFFLL);
   long long n_doc = 0;
-  {
-    long long v = threadIdx.x < kBins ? sh.tot[threadIdx.x] : 0;
-    n_doc = block_sum_ll(v, sh);
-  }
-  if (k > n_doc && rank == 0 && threadIdx.x == 0) tg::set_device_error(err, TG_DEVERR_K_GT_NDOC);
-  const long long K = k < n_doc ? k : n_doc;
-
-  // mode: 0 = keep no document token, 1 = keep all, 2 = radix threshold
-  const int mode = (K == 0) ? 0 : (K == n_doc ? 1 : 2);
-  uint32_t T = 0xFFFFFFFFu;  // keep key > T, plus the first need_eq keys == T in index order
+  int mode = 2;          // 0 = keep no document token, 1 = keep all, 2 = threshold
+  uint32_t T = 0u;       // keep key > T, plus the first need_eq keys == T in index order
   long long need_eq = 0;
-  if (mode == 1) {
-    T = 0u;  // every document key is > 0
-  } else if (mode == 2) {
-    uint32_t remaining = static_cast<uint32_t>(K);
-    select_digit(sh, remaining);
-    uint32_t prefix = sh.sel_digit << 24;
-    remaining -= sh.sel_above;
-    for (int pass = 1; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      cluster.sync();  // every CTA has finished reading the previous histograms
-      for (int b = threadIdx.x; b < kBins; b += kThreads) sh.hist[b] = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int buf = pass & 1;
+    const int shift = 24 - 8 * pass;
+    if (pass >= 2) {
+      // this buffer was read by every CTA before the cluster barrier of the previous pass
+      if (threadIdx.x < kBins) sh.hist[buf][threadIdx.x] = 0;
       __syncthreads();
-      const uint32_t hi_mask = 0xFFFFFFFFu << (shift + 8);
-      for (int i = threadIdx.x; i < m; i += kThreads) {
-        const uint32_t key = key_at(i);
-        if (key && (key & hi_mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 0xFFu], 1u);
-      }
-      __syncthreads();
-      cluster.sync();
-      cluster_sum_hist(cluster, sh);
-      select_digit(sh, remaining);
-      prefix |= sh.sel_digit << shift;
-      remaining -= sh.sel_above;
     }
-    T = prefix;
-    need_eq = remaining;
+    for (int rd = 0; rd < rounds; ++rd) {
+      if (!kResident) load_keys(rd);
+#pragma unroll
+      for (int e = 0; e < kItems; ++e)
+        if (keys[e] != 0u && (keys[e] & pmask) == prefix) atomicAdd(&sh.hist[buf][(keys[e] >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    cluster.sync();
+    cluster_select_digit(cluster, sh, buf, remaining);
+    if (pass == 0) {
+      n_doc = sh.wsum[kWarps];
+      if (k > n_doc && rank == 0 && threadIdx.x == 0) tg::set_device_error(err, TG_DEVERR_K_GT_NDOC);
+      if (k == 0 || n_doc == 0) { mode = 0; T = 0xFFFFFFFFu; break; }
+      if (k >= n_doc) { mode = 1; T = 0u; break; }
+    }
+    const uint32_t d = sh.sel_digit;
+    const uint32_t above = sh.sel_above, cnt = sh.sel_count;
+    prefix |= d << shift;
+    pmask |= 0xFFu << shift;
+    remaining -= above;
+    if (cnt == remaining) {
+      // every candidate of this bin is kept: threshold just below the bin
+      T = prefix ? prefix - 1u : 0u;  // (prefix = 0 would mean every document key is kept)
+      need_eq = 0;
+      break;
+    }
+    if (pass == 3) {
+      T = prefix;
+      need_eq = remaining;
+    }
   }
+  if (mode == 0) need_eq = 0;
 
-  // ---- exchange 1: ties (keys == T) per CTA, in index order across the cluster
-  long long c_eq = 0;
-  if (mode == 2) {
-    long long v = 0;
-    for (int i = threadIdx.x; i < m; i += kThreads) v += key_at(i) == T;
-    c_eq = block_sum_ll(v, sh);
+  // ---- per-thread counts: ties (key == T, threshold mode only) and certain keeps
+  // (question tokens and keys > T).  Within one round a CTA holds at most 16384
+  // positions, so the pair packs into one 32-bit value and one scan gives both prefixes.
+  auto count_round = [&](int rd, uint32_t &nt, uint32_t &ng) {
+    nt = 0;
+    ng = 0;
+#pragma unroll
+    for (int e = 0; e < kItems; ++e) {
+      if (!valid(rd, e)) continue;
+      nt += (mode == 2) && keys[e] == T;
+      ng += keys[e] == 0u || keys[e] > T;
+    }
+  };
+  uint32_t excl0 = 0, tot0 = 0;
+  long long cta_eq = 0, cta_gtq = 0;
+  if (kResident) {
+    uint32_t nt, ng;
+    count_round(0, nt, ng);
+    excl0 = block_excl_scan((nt << 16) | ng, sh, &tot0);
+    cta_eq = tot0 >> 16;
+    cta_gtq = tot0 & 0xFFFFu;
+  } else {
+    for (int rd = 0; rd < rounds; ++rd) {
+      load_keys(rd);
+      uint32_t nt, ng, t;
+      count_round(rd, nt, ng);
+      block_excl_scan((nt << 16) | ng, sh, &t);
+      cta_eq += t >> 16;
+      cta_gtq += t & 0xFFFFu;
+      __syncthreads();  // the next scan reuses the scan buffer
+    }
   }
-  if (threadIdx.x == 0) sh.exch[0] = c_eq;
+  if (threadIdx.x == 0) {
+    sh.exch[0] = cta_eq;
+    sh.exch[1] = cta_gtq;
+  }
   cluster.sync();
-  long long tie_base = 0;
-  for (int c = 0; c < rank; ++c) tie_base += cluster.map_shared_rank(sh.exch, c)[0];
-  long long ties_here = need_eq - tie_base;
-  ties_here = ties_here < 0 ? 0 : (ties_here > c_eq ? c_eq : ties_here);
-
-  // ---- exchange 2: kept count per CTA
-  long long c_keep = ties_here;
-  {
-    long long v = 0;
-    for (int i = threadIdx.x; i < m; i += kThreads) {
-      const uint32_t key = key_at(i);
-      v += (key == 0u) || (key > T);
+  if (threadIdx.x == 0) {
+    long long tb = 0, ob = base, nt = 0, my_tb = 0;
+    for (int r = 0; r < kCluster; ++r) {
+      const long long *x = cluster.map_shared_rank(&sh.exch[0], r);
+      const long long eq = x[0], gtq = x[1];
+      long long th = need_eq - tb;
+      th = th < 0 ? 0 : (th > eq ? eq : th);
+      if (r < rank) ob += gtq + th;
+      if (r == rank) my_tb = tb;
+      tb += eq;
+      nt += gtq + th;
     }
-    c_keep += block_sum_ll(v, sh);
+    sh.bcast[0] = my_tb;
+    sh.bcast[1] = ob;
+    if (!cu_seqlens && rank == 0) *n_kept = static_cast<int32_t>(nt);
+    if (cu_seqlens && rank == 0 && static_cast<long long>(cu_kept[seg + 1]) - base != nt)
+      tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
   }
-  if (threadIdx.x == 0) sh.exch[1] = c_keep;
-  cluster.sync();
-  long long out_base = base, n_total = 0;
-  for (int c = 0; c < kCluster; ++c) {
-    const long long v = cluster.map_shared_rank(sh.exch, c)[1];
-    if (c < rank) out_base += v;
-    n_total += v;
-  }
-  if (!cu_seqlens && rank == 0 && threadIdx.x == 0) *n_kept = static_cast<int32_t>(n_total);
-  if (cu_seqlens && rank == 0 && threadIdx.x == 0) {
-    if (static_cast<long long>(cu_kept[seg + 1]) - base != n_total) tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
-  }
+  __syncthreads();
+  const long long tie_base = sh.bcast[0], out_base = sh.bcast[1];
 
-  // ---- ordered compaction: tiles of kTile positions, kItems consecutive per thread
-  long long tie_run = 0, keep_run = 0;
-  for (int t0 = 0; t0 < m; t0 += kTile) {
-    uint32_t kk[kItems];
-    int n_tie = 0;
-#pragma unroll
-    for (int j = 0; j < kItems; ++j) {
-      const int i = t0 + threadIdx.x * kItems + j;
-      kk[j] = i < m ? key_at(i) : 0xFFFFFFFFu;  // out-of-range marker: never kept, never a tie
-      n_tie += (i < m) && (mode == 2) && (kk[j] == T);
+  // ---- ordered compaction.  The ties this CTA keeps are its first ``quota`` ties, so
+  // the kept ties before a thread are min(ties before it, quota).
+  long long quota = need_eq - tie_base;
+  quota = quota < 0 ? 0 : quota;
+  long long run_tie = 0, run_gtq = 0;
+  for (int rd = 0; rd < rounds; ++rd) {
+    uint32_t x = excl0, rt = tot0;
+    if (!kResident) {
+      load_keys(rd);
+      uint32_t nt, ng;
+      count_round(rd, nt, ng);
+      x = block_excl_scan((nt << 16) | ng, sh, &rt);
     }
-    int tie_tot = 0;
-    const int tie_excl = block_exclusive_scan(n_tie, sh.warp_tot, &tie_tot);
-    bool keep[kItems];
-    int n_keep = 0;
-    long long trank = tie_run + tie_excl;
+    long long trank = run_tie + (x >> 16);
+    long long pos = out_base + run_gtq + (x & 0xFFFFu) + (trank < quota ? trank : quota);
+    const int64_t p0 = lo + static_cast<int64_t>(rd) * kRound + static_cast<int64_t>(threadIdx.x) * kItems;
 #pragma unroll
-    for (int j = 0; j < kItems; ++j) {
-      const int i = t0 + threadIdx.x * kItems + j;
-      bool kp = false;
-      if (i < m) {
-        if (kk[j] == 0u || kk[j] > T) {
-          kp = true;
-        } else if (mode == 2 && kk[j] == T) {
-          kp = (tie_base + trank) < need_eq;
-          ++trank;
-        }
+    for (int e = 0; e < kItems; ++e) {
+      if (!valid(rd, e)) continue;
+      bool kp = keys[e] == 0u || keys[e] > T;
+      if (!kp && mode == 2 && keys[e] == T) {
+        kp = trank < quota;
+        ++trank;
       }
-      keep[j] = kp;
-      n_keep += kp;
-    }
-    int keep_tot = 0;
-    const int keep_excl = block_exclusive_scan(n_keep, sh.warp_tot, &keep_tot);
-    long long pos = out_base + keep_run + keep_excl;
-#pragma unroll
-    for (int j = 0; j < kItems; ++j) {
-      if (keep[j]) {
+      if (kp) {
         if (pos < cap) {
-          kept_idx[pos] = static_cast<int32_t>(lo + t0 + threadIdx.x * kItems + j);
+          kept_idx[pos] = static_cast<int32_t>(p0 + e);
         } else {
           tg::set_device_error(err, TG_DEVERR_CAPACITY);
         }
         ++pos;
       }
     }
-    tie_run += tie_tot;
-    keep_run += keep_tot;
+    run_tie += rt >> 16;
+    run_gtq += rt & 0xFFFFu;
+    if (!kResident) __syncthreads();  // the next round's scan reuses the scan buffer
   }
   cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
@@ -363,18 +393,19 @@ __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__rest
   }
 }
 
-tg_status configure() {
-  static bool done[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (!done[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kKeyCap * sizeof(uint32_t)));
-    if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    done[dev] = true;
-  }
-  return TG_OK;
+void launch_cluster(bool resident, unsigned grid, cudaStream_t s, const float *scores, const uint8_t *mask,
+                    int64_t n_single, int64_t k_single, const int32_t *cu, const int32_t *kps, const int32_t *cu_kept,
+                    int64_t total, int32_t *kept_idx, int64_t cap, int32_t *n_kept, uint32_t *err) {
+  if (resident)
+    topk_cluster_kernel<true><<<grid, kThreads, 0, s>>>(scores, mask, n_single, k_single, cu, kps, cu_kept, total,
+                                                         kept_idx, cap, n_kept, err);
+  else
+    topk_cluster_kernel<false><<<grid, kThreads, 0, s>>>(scores, mask, n_single, k_single, cu, kps, cu_kept, total,
+                                                          kept_idx, cap, n_kept, err);
 }
+
+// chunk per CTA for a request of ``len`` positions (as the kernel computes it)
+int64_t chunk_of(int64_t len) { return ((len + kCluster - 1) / kCluster + kItems - 1) / kItems * kItems; }
 
 }  // namespace
 
@@ -389,13 +420,8 @@ extern "C" tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask
   if (cap > 0 && !kept_idx) return tg::fail(TG_ERR_INVALID_ARG, "kept_idx is NULL");
   uint32_t *err = tg::device_error_word();
   if (!err) return TG_ERR_CUDA;
-  const int64_t chunk = (n + kCluster - 1) / kCluster;
-  const int use_cache = chunk <= kKeyCap;
-  const size_t smem = use_cache ? static_cast<size_t>(kKeyCap) * sizeof(uint32_t) : 0;
-  tg_status st = configure();
-  if (st != TG_OK) return st;
-  topk_cluster_kernel<<<kCluster, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      scores, doc_mask, n, k, nullptr, nullptr, nullptr, n, kept_idx, cap, n_kept, use_cache, err);
+  launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), scores, doc_mask, n, k, nullptr,
+                 nullptr, nullptr, n, kept_idx, cap, n_kept, err);
   return tg::check_launch("topk_cluster_kernel");
 }
 
@@ -417,12 +443,9 @@ extern "C" tg_status tg_select_topk_varlen(const float *scores, const uint8_t *d
   seg_offsets_kernel<<<1, 1024, 0, s>>>(doc_mask, cu_seqlens, B, total, k_per_seq, cu_kept, err);
   tg_status st = tg::check_launch("seg_offsets_kernel");
   if (st != TG_OK || B == 0) return st;
-  const int64_t chunk = (max_seqlen + kCluster - 1) / kCluster;
-  const int use_cache = chunk <= kKeyCap;
-  const size_t smem = use_cache ? static_cast<size_t>(kKeyCap) * sizeof(uint32_t) : 0;
-  st = configure();
-  if (st != TG_OK) return st;
-  topk_cluster_kernel<<<static_cast<unsigned>(B) * kCluster, kThreads, smem, s>>>(
-      scores, doc_mask, 0, 0, cu_seqlens, k_per_seq, cu_kept, total, kept_idx, cap, nullptr, use_cache, err);
+  // the resident variant is only chosen when every request's chunk fits; a request longer
+  // than max_seqlen would need the other variant, so max_seqlen must bound them all
+  launch_cluster(chunk_of(max_seqlen) <= kRound, static_cast<unsigned>(B) * kCluster, s, scores, doc_mask, 0, 0,
+                 cu_seqlens, k_per_seq, cu_kept, total, kept_idx, cap, nullptr, err);
   return tg::check_launch("topk_cluster_kernel");
 }

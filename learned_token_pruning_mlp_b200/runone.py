@@ -35,6 +35,7 @@ def main():
     ap.add_argument("--D", type=int, default=128)
     ap.add_argument("--tau", type=float, default=1.1)
     ap.add_argument("--repeat", type=int, default=3)
+    ap.add_argument("--graph", action="store_true", help="time a CUDA-graph replay of the calls")
     a = ap.parse_args()
     tgbuild.build()
     dev = torch.device("cuda:0")
@@ -74,10 +75,25 @@ def main():
     fn()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(a.repeat):
-        fn()
-    e1.record()
+    if a.graph:
+        # replay the calls from a CUDA graph so host-side call overhead does not leave the
+        # GPU idle between launches of a short kernel
+        stream = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(a.repeat):
+                    fn()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        graph.replay()
+        e1.record()
+    else:
+        e0.record()
+        for _ in range(a.repeat):
+            fn()
+        e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.repeat
     bits = tg.tg_get_device_error()
