@@ -8,15 +8,21 @@
 // B200 design.  At d = 2048, h = 256 the first layer is 2*d*h = 1 MFLOP per token
 // against 2*d = 4 KB of residual read once from HBM: 256 flop/B, right on the
 // B200 ridge (measured bf16 peak / measured HBM bandwidth ~ 250 flop/B).  CUDA-core
-// FMAs would be ~20x too slow, so the contraction runs on tcgen05:
-//   * persistent grid, one CTA per SM, tiles of 128 tokens (MMA M = 128, N = h);
-//   * warp 0 streams 128x64 residual tiles and the matching 64-wide slice of W1
-//     through a 4-stage TMA pipeline (128-byte swizzle, K-major operands);
-//   * warp 1 issues tcgen05.mma (one thread) into a TMEM accumulator of h fp32
-//     columns, double-buffered so the epilogue of tile t overlaps the MMAs of t+1;
-//   * warps 4-7 read the accumulator rows with tcgen05.ld (one token per thread)
-//     and apply +b1, SiLU, the dot with W2 and +b2 in registers, writing one fp32
-//     per token.  The hidden activations never leave the SM.
+// FMAs would be ~20x too slow, so the contraction runs on tcgen05.  A single-SM
+// M=128 x N=256 MMA reads 12 KB of operands from shared memory per 128 clocks while
+// TMA writes as much again, more than shared memory delivers, so the kernel runs on
+// CTA pairs (cta_group::2):
+//   * a 2-CTA cluster owns 256-token tiles: each CTA stages its 128 tokens x 64
+//     columns of the residual and its half (h/2 rows) of the matching 64-column
+//     slice of W1 (6 stages of 32 KB, 128-byte swizzle, K-major), both TMA loads
+//     completing on the pair leader's barrier;
+//   * the leader's warp 1 issues one tcgen05.mma.cta_group::2 (M = 256, N = h) per
+//     16 columns; each CTA's TMEM holds its 128 rows x h fp32 accumulator,
+//     double-buffered so the epilogue of tile t overlaps the MMAs of t+1.  W1 is
+//     now staged once per 256 tokens instead of once per 128;
+//   * warps 4-7 of each CTA read their accumulator rows with tcgen05.ld (one token
+//     per thread) and apply +b1, SiLU, the dot with W2 and +b2 in registers, writing
+//     one fp32 per token.  The hidden activations never leave the SM.
 // The residual is streamed with an L2 evict-first hint and W1 (re-read by every
 // tile) with evict-last, so W1 stays L2-resident while the residual passes through.
 #include <algorithm>
@@ -26,18 +32,18 @@
 
 namespace {
 
-constexpr int kBlockM = 128;
-constexpr int kBlockK = 64;  // bf16 elements in one 128-byte swizzled row
-constexpr int kStages = 4;
+constexpr int kBlockM = 128;      // tokens per CTA (256 per pair)
+constexpr int kBlockK = 64;       // bf16 elements in one 128-byte swizzled row
+constexpr int kStages = 6;
 constexpr int kThreads = 256;
 constexpr int kMaxH = 256;
-constexpr uint32_t kTileABytes = kBlockM * kBlockK * 2;
+constexpr uint32_t kTileABytes = kBlockM * kBlockK * 2;  // 16 KB
 
 struct GateCtl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t full[kStages];      // used in the leader: both CTAs' loads complete here
+  uint64_t empty[kStages];     // each CTA's own copy, signalled by the leader's MMA commit
+  uint64_t acc_full[2];        // each CTA's own copy
+  uint64_t acc_empty[2];       // used in the leader: 128 epilogue threads of each CTA
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -46,11 +52,11 @@ struct GateCtl {
 };
 
 constexpr size_t smem_bytes(int h) {
-  return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * (kTileABytes + static_cast<size_t>(h) * 128) +
+  return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * (kTileABytes + static_cast<size_t>(h / 2) * 128) +
          sizeof(GateCtl);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gate_score_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                       const __nv_bfloat16 *__restrict__ b1, const __nv_bfloat16 *__restrict__ W2,
                       const __nv_bfloat16 *__restrict__ b2, float *__restrict__ scores, int64_t n, int d, int h,
@@ -59,12 +65,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + kStages * kTileABytes;
-  const uint32_t tile_b_bytes = static_cast<uint32_t>(h) * 128u;
+  const uint32_t tile_b_bytes = static_cast<uint32_t>(h / 2) * 128u;  // this CTA's half of the W1 slice
   GateCtl *ctl = reinterpret_cast<GateCtl *>(sB + kStages * tile_b_bytes);
 
   const int warp = tg::warp_id();
   const int lane = threadIdx.x & 31;
-  const int64_t num_tiles = (n + kBlockM - 1) / kBlockM;
+  const uint32_t rank = tg::cluster_ctarank();       // 0 = leader, 1 = peer
+  const bool leader = rank == 0;
+  const int64_t pair = blockIdx.x >> 1;
+  const int64_t n_pairs = gridDim.x >> 1;
+  const int64_t num_tiles = (n + 2 * kBlockM - 1) / (2 * kBlockM);
   const int ksteps = (d + kBlockK - 1) / kBlockK;
 
   if (threadIdx.x == 0) {
@@ -74,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tg::mbar_init(tg::smem_addr(&ctl->acc_full[a]), 1);
-      tg::mbar_init(tg::smem_addr(&ctl->acc_empty[a]), 128);
+      tg::mbar_init(tg::smem_addr(&ctl->acc_empty[a]), 2 * 128);
     }
     tg::mbar_init(tg::smem_addr(&ctl->drain), 1);
     ctl->abort_flag = 0;
@@ -83,8 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::prefetch_tmap(&tm_w);
   }
   if (warp == 2) {
-    tg::tmem_alloc(tg::smem_addr(&ctl->tmem_base), tmem_cols);
-    tg::tmem_relinquish();
+    tg::tmem_alloc_pair(tg::smem_addr(&ctl->tmem_base), tmem_cols);
+    tg::tmem_relinquish_pair();
   }
   if (warp >= 4) {
     for (int j = threadIdx.x - 128; j < h; j += 128) {
@@ -92,35 +102,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctl->w2[j] = __bfloat162float(W2[j]);
     }
   }
+  // barriers of both CTAs initialised and TMEM allocated before any cross-CTA traffic
   tg::tc_fence_before();
   __syncthreads();
+  tg::cluster_sync_all();
   tg::tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int *abort_flag = &ctl->abort_flag;
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
     const uint64_t pol_x = tg::l2_policy_evict_first();
     const uint64_t pol_w = tg::l2_policy_evict_last();
     uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int64_t tile = pair; tile < num_tiles; tile += n_pairs) {
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
         const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
         if (!tg::mbar_wait(tg::smem_addr(&ctl->empty[s]), ph ^ 1u, abort_flag)) goto producer_done;
         const uint32_t full = tg::smem_addr(&ctl->full[s]);
-        tg::mbar_arrive_expect_tx(full, kTileABytes + tile_b_bytes);
-        tg::tma_load_2d_hint(tg::smem_addr(sA + s * kTileABytes), &tm_x, full, ks * kBlockK,
-                             static_cast<int32_t>(tile * kBlockM), pol_x);
-        tg::tma_load_2d_hint(tg::smem_addr(sB + s * tile_b_bytes), &tm_w, full, ks * kBlockK, 0, pol_w);
+        if (leader) tg::mbar_arrive_expect_tx(full, 2u * (kTileABytes + tile_b_bytes));
+        const uint32_t lbar = tg::pair_leader_addr(full);
+        tg::tma_load_2d_pair(tg::smem_addr(sA + s * kTileABytes), &tm_x, lbar, ks * kBlockK,
+                             static_cast<int32_t>(tile * 2 * kBlockM + rank * kBlockM), pol_x);
+        tg::tma_load_2d_pair(tg::smem_addr(sB + s * tile_b_bytes), &tm_w, lbar, ks * kBlockK,
+                             static_cast<int32_t>(rank * (h / 2)), pol_w);
       }
     }
   producer_done:;
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA issuer
-    const uint32_t idesc = tg::idesc_bf16_f32(kBlockM, h, false, false);
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------------------------------------------------------- MMA issuer (leader)
+    const uint32_t idesc = tg::idesc_bf16_f32(2 * kBlockM, h, false, false);
     uint32_t it = 0, tc = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
+    for (int64_t tile = pair; tile < num_tiles && ok; tile += n_pairs, ++tc) {
       const uint32_t acc = tc & 1u, aph = (tc >> 1) & 1u;
       if (!tg::mbar_wait(tg::smem_addr(&ctl->acc_empty[acc]), aph ^ 1u, abort_flag)) break;
       tg::tc_fence_after();
@@ -137,24 +151,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBlockK / 16; ++kk) {
           // advance 16 bf16 = 32 bytes along K inside the 128-byte swizzled rows
-          tg::mma_bf16_ss(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (ks | kk) != 0);
+          tg::mma_bf16_ss_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (ks | kk) != 0);
         }
-        tg::mma_commit(tg::smem_addr(&ctl->empty[s]));
+        tg::mma_commit_pair_multicast(tg::smem_addr(&ctl->empty[s]), 0x3);
       }
-      if (ok) tg::mma_commit(tg::smem_addr(&ctl->acc_full[acc]));
+      if (ok) tg::mma_commit_pair_multicast(tg::smem_addr(&ctl->acc_full[acc]), 0x3);
     }
     if (*abort_flag) {
       // let every MMA already issued finish before TMEM is released
-      tg::mma_commit(tg::smem_addr(&ctl->drain));
+      tg::mma_commit_pair_multicast(tg::smem_addr(&ctl->drain), 0x1);
       int local_abort = 0;
       tg::mbar_wait(tg::smem_addr(&ctl->drain), 0, &local_abort, 100000000ull);
     }
   } else if (warp >= 4) {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue (both CTAs)
     const int quarter = warp - 4;  // TMEM lanes 32*quarter .. 32*quarter+31
     const float bias2 = __bfloat162float(b2[0]);
     uint32_t tc = 0;
-    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+    for (int64_t tile = pair; tile < num_tiles; tile += n_pairs, ++tc) {
       const uint32_t acc = tc & 1u, aph = (tc >> 1) & 1u;
       if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->acc_full[acc]), aph, abort_flag)) break;
       tg::tc_fence_after();
@@ -172,18 +186,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tg::tc_fence_before();
-      tg::mbar_arrive(tg::smem_addr(&ctl->acc_empty[acc]));
-      const int64_t row = tile * kBlockM + quarter * 32 + lane;
+      tg::mbar_arrive_remote(tg::smem_addr(&ctl->acc_empty[acc]), 0u);  // the leader's copy
+      const int64_t row = tile * 2 * kBlockM + rank * kBlockM + quarter * 32 + lane;
       if (row < n) scores[row] = sum + bias2;
     }
   }
 
+  // every MMA, remote arrive and peer TMEM access is done before either CTA frees TMEM
   tg::tc_fence_before();
   __syncthreads();
+  tg::cluster_sync_all();
   if (threadIdx.x == 0 && ctl->abort_flag) tg::set_device_error(err, TG_DEVERR_TIMEOUT);
   if (warp == 2) {
     tg::tc_fence_after();
-    tg::tmem_dealloc(tmem_base, tmem_cols);
+    tg::tmem_dealloc_pair(tmem_base, tmem_cols);
   }
 }
 
@@ -216,7 +232,7 @@ extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, 
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(h)};
     const uint64_t strides[1] = {static_cast<uint64_t>(d) * 2};
-    const uint32_t box[2] = {kBlockK, static_cast<uint32_t>(h)};
+    const uint32_t box[2] = {kBlockK, static_cast<uint32_t>(h / 2)};
     if (!tg::encode_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W1, dims, strides, box,
                          CU_TENSOR_MAP_SWIZZLE_128B))
       return TG_ERR_CUDA;
@@ -234,9 +250,9 @@ extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, 
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     configured[dev] = true;
   }
-  const int64_t num_tiles = (n + kBlockM - 1) / kBlockM;
-  const int grid = static_cast<int>(std::min<int64_t>(num_tiles, tg::sm_count()));
-  gate_score_kernel<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+  const int64_t num_tiles = (n + 2 * kBlockM - 1) / (2 * kBlockM);
+  const int64_t pairs = std::min<int64_t>(num_tiles, tg::sm_count() / 2);
+  gate_score_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       tm_x, tm_w, reinterpret_cast<const __nv_bfloat16 *>(b1), reinterpret_cast<const __nv_bfloat16 *>(W2),
       reinterpret_cast<const __nv_bfloat16 *>(b2), scores, n, d, h, tmem_cols, err);
   return tg::check_launch("gate_score_kernel");
