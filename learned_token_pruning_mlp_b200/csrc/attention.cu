@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sQx = sV + NS * C::kTileBytes;              // [128 x 16] block of ones (columns 0, 1)
   uint8_t *sKx = sQx + kExtBytes;                      // [NS][128 x 16] blocks of c_j (columns 0, 1)
   AttnCtl *ctl = reinterpret_cast<AttnCtl *>(sKx + NS * kExtBytes);
+  tg::pdl_wait();
+  tg::pdl_trigger();
 
   // ---- work unit: heaviest query blocks first, then request, then head
   const int per_mb = Hq * B;
@@ -437,9 +439,11 @@ tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const fl
   const int64_t grid = static_cast<int64_t>(n_mblocks) * Hq * B;
   if (grid == 0) return TG_OK;
   if (grid > 0x7FFFFFFFLL) return tg::fail(TG_ERR_UNSUPPORTED, "grid too large");
-  gated_attention_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(
-      tm_q, tm_k, tm_v, s, gain, scale_log2, cu_seqlens, cu_seqlens ? 0 : total, total, n_mblocks, B, Hq, Hkv,
-      reinterpret_cast<__nv_bfloat16 *>(O), err);
+  const cudaError_t e = tg::launch_pdl(gated_attention_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+                                      C::kSmem, stream, tm_q, tm_k, tm_v, s, gain, scale_log2, cu_seqlens,
+                                      cu_seqlens ? int64_t(0) : total, total, n_mblocks, B, Hq, Hkv,
+                                      reinterpret_cast<__nv_bfloat16 *>(O), err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gated_attention_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("gated_attention_kernel");
 }
 

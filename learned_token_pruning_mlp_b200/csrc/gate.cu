@@ -96,17 +96,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tg::tmem_alloc_pair(tg::smem_addr(&ctl->tmem_base), tmem_cols);
     tg::tmem_relinquish_pair();
   }
-  if (warp >= 4) {
-    for (int j = threadIdx.x - 128; j < h; j += 128) {
-      ctl->b1[j] = __bfloat162float(b1[j]);
-      ctl->w2[j] = __bfloat162float(W2[j]);
-    }
-  }
   // barriers of both CTAs initialised and TMEM allocated before any cross-CTA traffic
   tg::tc_fence_before();
   __syncthreads();
   tg::cluster_sync_all();
   tg::tc_fence_after();
+  // the prologue above overlaps the previous kernel; global memory only from here on
+  tg::pdl_wait();
+  tg::pdl_trigger();
+  if (warp >= 4) {
+    for (int j = threadIdx.x - 128; j < h; j += 128) {
+      ctl->b1[j] = __bfloat162float(b1[j]);
+      ctl->w2[j] = __bfloat162float(W2[j]);
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+  }
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int *abort_flag = &ctl->abort_flag;
 
@@ -252,8 +256,11 @@ extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, 
   }
   const int64_t num_tiles = (n + 2 * kBlockM - 1) / (2 * kBlockM);
   const int64_t pairs = std::min<int64_t>(num_tiles, tg::sm_count() / 2);
-  gate_score_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      tm_x, tm_w, reinterpret_cast<const __nv_bfloat16 *>(b1), reinterpret_cast<const __nv_bfloat16 *>(W2),
-      reinterpret_cast<const __nv_bfloat16 *>(b2), scores, n, d, h, tmem_cols, err);
+  const cudaError_t e = tg::launch_pdl(gate_score_kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem,
+                                      static_cast<cudaStream_t>(stream), tm_x, tm_w,
+                                      reinterpret_cast<const __nv_bfloat16 *>(b1),
+                                      reinterpret_cast<const __nv_bfloat16 *>(W2),
+                                      reinterpret_cast<const __nv_bfloat16 *>(b2), scores, n, d, h, tmem_cols, err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gate_score_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("gate_score_kernel");
 }

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(
     const float *__restrict__ scores, float *__restrict__ s_k, int stages, uint32_t *err) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int abort_flag;
+  tg::pdl_wait();
+  tg::pdl_trigger();
 
   int64_t rows = n_rows;
   if (n_kept_dev) {
@@ -126,8 +128,10 @@ extern "C" tg_status tg_gather(const tg_bf16 *hidden, int64_t n, int32_t d, cons
   const int64_t warps_needed = (n_rows + stages - 1) / stages;
   int64_t grid = (warps_needed + kWarps - 1) / kWarps;
   grid = std::max<int64_t>(1, std::min<int64_t>(grid, 2LL * tg::sm_count()));
-  gather_rows_kernel<<<static_cast<unsigned>(grid), kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint8_t *>(hidden), n, row_bytes, kept_idx, n_rows, n_kept,
-      reinterpret_cast<uint8_t *>(hidden_k), scores, s_k, stages, err);
+  const cudaError_t e = tg::launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
+                                      static_cast<cudaStream_t>(stream), reinterpret_cast<const uint8_t *>(hidden), n,
+                                      row_bytes, kept_idx, n_rows, n_kept, reinterpret_cast<uint8_t *>(hidden_k),
+                                      scores, s_k, stages, err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gather_rows_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("gather_rows_kernel");
 }

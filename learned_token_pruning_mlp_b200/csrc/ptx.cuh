@@ -84,6 +84,14 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, vo
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched so that it may start while the preceding
+// kernel on the stream finishes; it calls pdl_wait() before its first global-memory
+// access (which returns once that kernel has completed and its writes are visible)
+// and pdl_trigger() to let the next kernel begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -149,6 +149,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
                         const int32_t *__restrict__ cu_kept, int64_t total, int32_t *__restrict__ kept_idx,
                         int64_t cap, int32_t *__restrict__ n_kept, uint32_t *err) {
   __shared__ TopkShared sh;
+  tg::pdl_wait();
+  tg::pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int seg = static_cast<int>(blockIdx.x) / kCluster;
@@ -257,32 +259,32 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   if (mode == 0) need_eq = 0;
 
   // ---- per-thread counts: ties (key == T, threshold mode only) and certain keeps
-  // (question tokens and keys > T).  Within one round a CTA holds at most 16384
-  // positions, so the pair packs into one 32-bit value and one scan gives both prefixes.
-  auto count_round = [&](int rd, uint32_t &nt, uint32_t &ng) {
-    nt = 0;
-    ng = 0;
+  // (question tokens and keys > T), kept as 16-bit masks of the thread's positions.
+  // Within one round a CTA holds at most 16384 positions, so the two counts pack into
+  // one 32-bit value and one block scan gives both prefixes.
+  auto classify = [&](int rd, uint32_t &tie_bits, uint32_t &keep_bits) {
+    tie_bits = 0;
+    keep_bits = 0;
 #pragma unroll
     for (int e = 0; e < kItems; ++e) {
-      if (!valid(rd, e)) continue;
-      nt += (mode == 2) && keys[e] == T;
-      ng += keys[e] == 0u || keys[e] > T;
+      const bool v = valid(rd, e);
+      tie_bits |= static_cast<uint32_t>(v && mode == 2 && keys[e] == T) << e;
+      keep_bits |= static_cast<uint32_t>(v && (keys[e] == 0u || keys[e] > T)) << e;
     }
   };
-  uint32_t excl0 = 0, tot0 = 0;
+  uint32_t tie_bits0 = 0, keep_bits0 = 0, excl0 = 0, tot0 = 0;
   long long cta_eq = 0, cta_gtq = 0;
   if (kResident) {
-    uint32_t nt, ng;
-    count_round(0, nt, ng);
-    excl0 = block_excl_scan((nt << 16) | ng, sh, &tot0);
+    classify(0, tie_bits0, keep_bits0);
+    excl0 = block_excl_scan((static_cast<uint32_t>(__popc(tie_bits0)) << 16) | __popc(keep_bits0), sh, &tot0);
     cta_eq = tot0 >> 16;
     cta_gtq = tot0 & 0xFFFFu;
   } else {
     for (int rd = 0; rd < rounds; ++rd) {
       load_keys(rd);
-      uint32_t nt, ng, t;
-      count_round(rd, nt, ng);
-      block_excl_scan((nt << 16) | ng, sh, &t);
+      uint32_t tb, kb, t;
+      classify(rd, tb, kb);
+      block_excl_scan((static_cast<uint32_t>(__popc(tb)) << 16) | __popc(kb), sh, &t);
       cta_eq += t >> 16;
       cta_gtq += t & 0xFFFFu;
       __syncthreads();  // the next scan reuses the scan buffer
@@ -293,23 +295,41 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     sh.exch[1] = cta_gtq;
   }
   cluster.sync();
-  if (threadIdx.x == 0) {
-    long long tb = 0, ob = base, nt = 0, my_tb = 0;
-    for (int r = 0; r < kCluster; ++r) {
-      const long long *x = cluster.map_shared_rank(&sh.exch[0], r);
-      const long long eq = x[0], gtq = x[1];
-      long long th = need_eq - tb;
-      th = th < 0 ? 0 : (th > eq ? eq : th);
-      if (r < rank) ob += gtq + th;
-      if (r == rank) my_tb = tb;
-      tb += eq;
-      nt += gtq + th;
+  if (threadIdx.x < 32) {
+    // lane r < 8 reads CTA r's counts; the prefixes over CTAs come from warp shuffles
+    const int lane = threadIdx.x;
+    long long eq = 0, gtq = 0;
+    if (lane < kCluster) {
+      const long long *x = cluster.map_shared_rank(&sh.exch[0], lane);
+      eq = x[0];
+      gtq = x[1];
     }
-    sh.bcast[0] = my_tb;
-    sh.bcast[1] = ob;
-    if (!cu_seqlens && rank == 0) *n_kept = static_cast<int32_t>(nt);
-    if (cu_seqlens && rank == 0 && static_cast<long long>(cu_kept[seg + 1]) - base != nt)
-      tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
+    long long eq_incl = eq;
+#pragma unroll
+    for (int off = 1; off < kCluster; off <<= 1) {
+      const long long t = __shfl_up_sync(0xFFFFFFFFu, eq_incl, off);
+      if (lane >= off) eq_incl += t;
+    }
+    const long long tb = eq_incl - eq;  // ties in CTAs before this lane's CTA
+    long long th = need_eq - tb;
+    th = th < 0 ? 0 : (th > eq ? eq : th);
+    const long long keep = lane < kCluster ? gtq + th : 0;
+    long long keep_incl = keep;
+#pragma unroll
+    for (int off = 1; off < kCluster; off <<= 1) {
+      const long long t = __shfl_up_sync(0xFFFFFFFFu, keep_incl, off);
+      if (lane >= off) keep_incl += t;
+    }
+    const long long nt = __shfl_sync(0xFFFFFFFFu, keep_incl, kCluster - 1);
+    if (lane == rank) {
+      sh.bcast[0] = tb;
+      sh.bcast[1] = base + keep_incl - keep;
+    }
+    if (lane == 0) {
+      if (!cu_seqlens && rank == 0) *n_kept = static_cast<int32_t>(nt);
+      if (cu_seqlens && rank == 0 && static_cast<long long>(cu_kept[seg + 1]) - base != nt)
+        tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
+    }
   }
   __syncthreads();
   const long long tie_base = sh.bcast[0], out_base = sh.bcast[1];
@@ -320,32 +340,34 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   quota = quota < 0 ? 0 : quota;
   long long run_tie = 0, run_gtq = 0;
   for (int rd = 0; rd < rounds; ++rd) {
-    uint32_t x = excl0, rt = tot0;
+    uint32_t x = excl0, rt = tot0, tie_bits = tie_bits0, keep_bits = keep_bits0;
     if (!kResident) {
       load_keys(rd);
-      uint32_t nt, ng;
-      count_round(rd, nt, ng);
-      x = block_excl_scan((nt << 16) | ng, sh, &rt);
+      classify(rd, tie_bits, keep_bits);
+      x = block_excl_scan((static_cast<uint32_t>(__popc(tie_bits)) << 16) | __popc(keep_bits), sh, &rt);
     }
-    long long trank = run_tie + (x >> 16);
-    long long pos = out_base + run_gtq + (x & 0xFFFFu) + (trank < quota ? trank : quota);
+    // kept ties of this thread: the first (quota - ties before it) of its tie positions
+    const long long tbefore = run_tie + (x >> 16);
+    long long allow = quota - tbefore;
+    allow = allow < 0 ? 0 : (allow > 16 ? 16 : allow);
+    uint32_t tb = 0, rem = tie_bits;
+    for (long long c = 0; c < allow && rem; ++c) {  // keep the lowest ``allow`` tie positions
+      tb |= rem & (~rem + 1u);
+      rem &= rem - 1u;
+    }
+    const uint32_t out_bits = keep_bits | tb;
+    long long pos = out_base + run_gtq + (x & 0xFFFFu) + (tbefore < quota ? tbefore : quota);
     const int64_t p0 = lo + static_cast<int64_t>(rd) * kRound + static_cast<int64_t>(threadIdx.x) * kItems;
-#pragma unroll
-    for (int e = 0; e < kItems; ++e) {
-      if (!valid(rd, e)) continue;
-      bool kp = keys[e] == 0u || keys[e] > T;
-      if (!kp && mode == 2 && keys[e] == T) {
-        kp = trank < quota;
-        ++trank;
+    uint32_t bits = out_bits;
+    while (bits) {
+      const int e = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (pos < cap) {
+        kept_idx[pos] = static_cast<int32_t>(p0 + e);
+      } else {
+        tg::set_device_error(err, TG_DEVERR_CAPACITY);
       }
-      if (kp) {
-        if (pos < cap) {
-          kept_idx[pos] = static_cast<int32_t>(p0 + e);
-        } else {
-          tg::set_device_error(err, TG_DEVERR_CAPACITY);
-        }
-        ++pos;
-      }
+      ++pos;
     }
     run_tie += rt >> 16;
     run_gtq += rt & 0xFFFFu;
@@ -362,6 +384,8 @@ __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__rest
                                                            int32_t *__restrict__ cu_kept, uint32_t *err) {
   __shared__ long long red[32];
   __shared__ long long run;
+  tg::pdl_wait();
+  tg::pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     run = 0;
@@ -393,15 +417,15 @@ __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__rest
   }
 }
 
-void launch_cluster(bool resident, unsigned grid, cudaStream_t s, const float *scores, const uint8_t *mask,
-                    int64_t n_single, int64_t k_single, const int32_t *cu, const int32_t *kps, const int32_t *cu_kept,
-                    int64_t total, int32_t *kept_idx, int64_t cap, int32_t *n_kept, uint32_t *err) {
+cudaError_t launch_cluster(bool resident, unsigned grid, cudaStream_t s, const float *scores, const uint8_t *mask,
+                           int64_t n_single, int64_t k_single, const int32_t *cu, const int32_t *kps,
+                           const int32_t *cu_kept, int64_t total, int32_t *kept_idx, int64_t cap, int32_t *n_kept,
+                           uint32_t *err) {
   if (resident)
-    topk_cluster_kernel<true><<<grid, kThreads, 0, s>>>(scores, mask, n_single, k_single, cu, kps, cu_kept, total,
-                                                         kept_idx, cap, n_kept, err);
-  else
-    topk_cluster_kernel<false><<<grid, kThreads, 0, s>>>(scores, mask, n_single, k_single, cu, kps, cu_kept, total,
-                                                          kept_idx, cap, n_kept, err);
+    return tg::launch_pdl(topk_cluster_kernel<true>, dim3(grid), dim3(kThreads), 0, s, scores, mask, n_single, k_single,
+                          cu, kps, cu_kept, total, kept_idx, cap, n_kept, err);
+  return tg::launch_pdl(topk_cluster_kernel<false>, dim3(grid), dim3(kThreads), 0, s, scores, mask, n_single, k_single,
+                        cu, kps, cu_kept, total, kept_idx, cap, n_kept, err);
 }
 
 // chunk per CTA for a request of ``len`` positions (as the kernel computes it)
@@ -420,8 +444,9 @@ extern "C" tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask
   if (cap > 0 && !kept_idx) return tg::fail(TG_ERR_INVALID_ARG, "kept_idx is NULL");
   uint32_t *err = tg::device_error_word();
   if (!err) return TG_ERR_CUDA;
-  launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), scores, doc_mask, n, k, nullptr,
-                 nullptr, nullptr, n, kept_idx, cap, n_kept, err);
+  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), scores,
+                                      doc_mask, n, k, nullptr, nullptr, nullptr, n, kept_idx, cap, n_kept, err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
 
@@ -440,12 +465,15 @@ extern "C" tg_status tg_select_topk_varlen(const float *scores, const uint8_t *d
   uint32_t *err = tg::device_error_word();
   if (!err) return TG_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  seg_offsets_kernel<<<1, 1024, 0, s>>>(doc_mask, cu_seqlens, B, total, k_per_seq, cu_kept, err);
+  cudaError_t e = tg::launch_pdl(seg_offsets_kernel, dim3(1), dim3(1024), 0, s, doc_mask, cu_seqlens, B, total,
+                                 k_per_seq, cu_kept, err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "seg_offsets_kernel launch: %s", cudaGetErrorString(e));
   tg_status st = tg::check_launch("seg_offsets_kernel");
   if (st != TG_OK || B == 0) return st;
   // the resident variant is only chosen when every request's chunk fits; a request longer
   // than max_seqlen would need the other variant, so max_seqlen must bound them all
-  launch_cluster(chunk_of(max_seqlen) <= kRound, static_cast<unsigned>(B) * kCluster, s, scores, doc_mask, 0, 0,
-                 cu_seqlens, k_per_seq, cu_kept, total, kept_idx, cap, nullptr, err);
+  e = launch_cluster(chunk_of(max_seqlen) <= kRound, static_cast<unsigned>(B) * kCluster, s, scores, doc_mask, 0, 0,
+                     cu_seqlens, k_per_seq, cu_kept, total, kept_idx, cap, nullptr, err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
