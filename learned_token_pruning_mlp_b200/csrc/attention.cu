@@ -29,8 +29,9 @@
 //     be issued right after O_t += P_t(j) V_j even though it overwrites P_t(j).
 //   * warps 4-7 and 8-11 are the softmax warpgroups of tile 0 and tile 1 (one query
 //     row per thread): tcgen05.ld of the S' row, causal mask on the diagonal tile,
-//     8-way max, exp2 of one packed f32x2 FMA per pair, 8-way sum, bf16 pack,
-//     tcgen05.st of P.  While one warpgroup works on its softmax the tensor core
+//     8-way max, exp2 of one packed f32x2 FMA per pair, bf16 pack, 8-way sum of the
+//     rounded weights with mixed-precision adds (so normalisation matches the
+//     weights the PV product uses), tcgen05.st of P.  While one warpgroup works on its softmax the tensor core
 //     works on the other tile's products.
 //   * The running max is only moved when it grows by more than 2^8 for some row of
 //     the warp (decided per warp: TMEM access is warp-collective); then O_t is
@@ -173,6 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int *abort_flag = &ctl->abort_flag;
 
+  // Register split: the launch gives 384 threads x 168 registers; the loader/MMA
+  // warpgroup needs few, the two softmax warpgroups hold a 128-wide S row each.
+  // 128 x 56 + 256 x 224 = 384 x 168, so the increase never waits.  Each warpgroup
+  // changes its budget inside its own branch.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
     const int nq = n1 ? 2 : 1;
@@ -291,7 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int local_abort = 0;
       tg::mbar_wait(tg::smem_addr(&ctl->drain), 0, &local_abort, 100000000ull);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
     // ------------------------------------------------------------ softmax + epilogue
     const int t = (warp - 4) >> 2;          // query tile of this warpgroup
     const int quarter = warp & 3;           // TMEM lane quarter
@@ -338,24 +347,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float nms = -m * eff;
       const uint64_t nms2 = tg::f2_pack(nms, nms);
-      uint64_t acc[4] = {0, 0, 0, 0};
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kBN / 2; ++c) {
         const uint64_t arg = tg::f2_fma(tg::f2_pack(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), eff2, nms2);
         float a0, a1;
         tg::f2_unpack(arg, a0, a1);
-        const float p0 = tg::ex2_approx(a0), p1 = tg::ex2_approx(a1);
-        acc[c & 3] = tg::f2_add(acc[c & 3], tg::f2_pack(p0, p1));
-        x[c] = pack_bf16x2(p0, p1);  // in place: x[c] is no longer needed once read above
+        const uint32_t pb = pack_bf16x2(tg::ex2_approx(a0), tg::ex2_approx(a1));
+        x[c] = pb;  // in place: x[c] is no longer needed once read above
+        // the row sum adds the same bf16-rounded weights the PV product uses, so every
+        // output row is an exact convex combination of its value rows
+        tg::add_bf16x2_to_f32(acc[(2 * c) & 7], acc[(2 * c + 1) & 7], pb);
       }
       tg::tmem_st32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
       tg::tmem_st32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-      float s0, s1, s2, s3, s4, s5, s6, s7;
-      tg::f2_unpack(acc[0], s0, s1);
-      tg::f2_unpack(acc[1], s2, s3);
-      tg::f2_unpack(acc[2], s4, s5);
-      tg::f2_unpack(acc[3], s6, s7);
-      l = fmaf(l, alpha, ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+      l = fmaf(l, alpha, ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
       if (rescale && j > 0) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
