@@ -274,6 +274,10 @@ def test_attention_full_size_sampled_rows():
 
 # =============================================================================== pipeline
 def test_pipeline_tiny_and_pruned_tokens_never_influence():
+    """The whole path on the tiny workload.  Each GPU stage is compared with the oracle
+    on inputs that come from the oracle side only (its fp32 gate scores and kept
+    indices); the all-GPU chain is checked for the article's structural properties and
+    for pruned positions never influencing any output."""
     w = W.get("tiny_n512")
     hidden, W1, b1, W2, b2 = W.gate_inputs(w)
     mask = W.doc_mask(w)
@@ -281,53 +285,57 @@ def test_pipeline_tiny_and_pruned_tokens_never_influence():
     Qf, Kf, Vf = W.attention_inputs(w, N)
     gain, tau = W.attention_params(w)
     k = w.segments[0].k
+    q = w.segments[0].q
+    d_gate = [t.to(DEV) for t in (W1, b1, W2, b2)]
 
-    def run(hid, Qa, Ka, Va):
-        d = [t.to(DEV) for t in (hid, W1, b1, W2, b2)]
-        scores = tg.tg_gate_score(*d)
-        kept, n_kept = tg.tg_select_topk(scores, mask.to(DEV), k)
-        S = int(n_kept.item())
-        kept = kept[:S].contiguous()
-        hk, sk = tg.tg_gather(d[0], kept, scores=scores)
-        kc = kept.long()
-        O = tg.tg_gated_attention(Qa.to(DEV)[kc].contiguous(), Ka.to(DEV)[kc].contiguous(),
-                                  Va.to(DEV)[kc].contiguous(), sk, gain.to(DEV), tau)
-        return scores.cpu(), kept.cpu(), hk.cpu(), sk.cpu(), O.cpu()
-
-    scores, kept, hk, sk, O = run(hidden, Qf, Kf, Vf)
+    # stage by stage against the oracle
+    scores = tg.tg_gate_score(hidden.to(DEV), *d_gate)
     ref_scores = oracle.gate_score(hidden, W1, b1, W2, b2)
-    assert_gate_close(scores.numpy(), ref_scores)
-    ref_kept = oracle.select_topk(scores.numpy(), mask, k)          # same fp32 array: bit-exact
-    assert np.array_equal(kept.numpy(), ref_kept)
-    assert len(ref_kept) == k + w.segments[0].q
-    ref_hk, ref_sk = oracle.gather(hidden, ref_kept, scores)
-    assert np.array_equal(hk.view(torch.int16).numpy().view(np.uint16), ref_hk)
+    assert_gate_close(scores.cpu().numpy(), ref_scores)
+    shared = ref_scores.astype(np.float32)
+    ref_kept = oracle.select_topk(shared, mask, k)
+    assert len(ref_kept) == k + q
+    kept, n_kept = tg.tg_select_topk(torch.as_tensor(shared).to(DEV), mask.to(DEV), k)
+    assert int(n_kept.item()) == len(ref_kept)
+    assert np.array_equal(kept[:len(ref_kept)].cpu().numpy(), ref_kept)
+    hk, sk = tg.tg_gather(hidden.to(DEV), torch.as_tensor(ref_kept).to(DEV), scores=torch.as_tensor(shared).to(DEV))
+    ref_hk, ref_sk = oracle.gather(hidden, ref_kept, shared)
+    assert np.array_equal(hk.cpu().view(torch.int16).numpy().view(np.uint16), ref_hk)
+    assert np.array_equal(sk.cpu().numpy(), ref_sk)
     kc = torch.as_tensor(ref_kept).long()
-    ref_O = oracle.gated_attention(Qf[kc], Kf[kc], Vf[kc], ref_sk, gain, tau)
-    assert_attn_close(O.float().numpy(), ref_O)
+    O = tg.tg_gated_attention(Qf[kc].contiguous().to(DEV), Kf[kc].contiguous().to(DEV), Vf[kc].contiguous().to(DEV),
+                              torch.as_tensor(ref_sk).to(DEV), gain.to(DEV), tau)
+    assert_attn_close(O.float().cpu().numpy(), oracle.gated_attention(Qf[kc], Kf[kc], Vf[kc], ref_sk, gain, tau))
 
-    # poison every pruned position of the full-length inputs: outputs stay bitwise equal
-    pruned = torch.as_tensor(np.setdiff1d(np.arange(N), ref_kept)).long()
+    # the all-GPU chain
+    def run(hid, Qa, Ka, Va, poison=None):
+        d = hid.to(DEV)
+        sc = tg.tg_gate_score(hidden.to(DEV), *d_gate)  # scoring sees the real residual
+        kp, nk = tg.tg_select_topk(sc, mask.to(DEV), k)
+        kp = kp[:int(nk.item())].contiguous()
+        if poison is not None:
+            sc = sc.clone()
+            sc[poison.to(DEV)] = float("nan")
+        hk2, sk2 = tg.tg_gather(d, kp, scores=sc)
+        kl = kp.long()
+        O2 = tg.tg_gated_attention(Qa.to(DEV)[kl].contiguous(), Ka.to(DEV)[kl].contiguous(),
+                                   Va.to(DEV)[kl].contiguous(), sk2, gain.to(DEV), tau)
+        return kp.cpu(), hk2.cpu(), O2.cpu()
+
+    kp, hk_g, O_g = run(hidden, Qf, Kf, Vf)
+    kept_np = kp.numpy()
+    assert len(kept_np) == k + q and np.all(np.diff(kept_np) > 0)
+    assert set(range(N - q, N)) <= set(kept_np.tolist())
+    # poison every position the GPU chain pruned: outputs stay bitwise equal and NaN-free
+    pruned = torch.as_tensor(np.setdiff1d(np.arange(N), kept_np)).long()
     hp, Qp, Kp, Vp = hidden.clone(), Qf.clone(), Kf.clone(), Vf.clone()
-    # the gate must still see the real residuals to reproduce the same selection, so the
-    # residual is poisoned only for the gather (after scoring) and Q/K/V fully
-    d = [t.to(DEV) for t in (hidden, W1, b1, W2, b2)]
-    sc = tg.tg_gate_score(*d)
-    kept2, n2 = tg.tg_select_topk(sc, mask.to(DEV), k)
-    kept2 = kept2[:int(n2.item())].contiguous()
-    hp[pruned] = float("nan")
-    Qp[pruned] = float("nan")
-    Kp[pruned] = float("nan")
-    Vp[pruned] = float("nan")
-    scp = sc.clone()
-    scp[pruned.to(DEV)] = float("nan")
-    hk2, sk2 = tg.tg_gather(hp.to(DEV), kept2, scores=scp)
-    k2 = kept2.long()
-    O2 = tg.tg_gated_attention(Qp.to(DEV)[k2].contiguous(), Kp.to(DEV)[k2].contiguous(), Vp.to(DEV)[k2].contiguous(),
-                               sk2, gain.to(DEV), tau)
-    assert torch.equal(hk2.cpu().view(torch.int16), hk.view(torch.int16))
-    assert torch.equal(O2.cpu().view(torch.int16), O.view(torch.int16))
-    assert not torch.isnan(O2.float()).any()
+    for t in (hp, Qp, Kp, Vp):
+        t[pruned] = float("nan")
+    kp2, hk_p, O_p = run(hp, Qp, Kp, Vp, poison=pruned)
+    assert torch.equal(kp2, kp)
+    assert torch.equal(hk_p.view(torch.int16), hk_g.view(torch.int16))
+    assert torch.equal(O_p.view(torch.int16), O_g.view(torch.int16))
+    assert not torch.isnan(O_p.float()).any()
 
 
 # =============================================================================== failure path
