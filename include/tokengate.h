@@ -137,12 +137,34 @@ tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask, int64_t n
  * kept_idx[cu_kept[b] .. cu_kept[b+1]) and cu_kept (device int32 [B+1]) is
  * written with cu_kept[0] = 0.  max_seqlen is a host upper bound on any
  * request's length and total the packed length (the bound cu_seqlens must
- * respect).  Malformed cu_seqlens set TG_DEVERR_BAD_SEQLENS. */
+ * respect).  Malformed cu_seqlens, or a request longer than max_seqlen, set
+ * TG_DEVERR_BAD_SEQLENS (the kept indices are then invalid). */
 tg_status tg_select_topk_varlen(const float *scores, const uint8_t *doc_mask,
                                 const int32_t *cu_seqlens, int32_t B, int64_t total,
                                 const int32_t *k_per_seq, int64_t max_seqlen,
                                 int32_t *kept_idx, int64_t cap, int32_t *cu_kept,
                                 tg_stream stream);
+
+/* Budget sweep: the same selection for m budgets in one launch (one thread-block
+ * cluster per budget), e.g. for the accuracy-versus-budget curves of the TokenGate
+ * article ("How does TokenGate perform on benchmarks?") or a training step's random
+ * budget ("What is token-gated attention?").  ks: device int32 [m]; budget b's kept
+ * indices go to kept_idx[b * stride ...] (capacity stride each) and its count to
+ * n_kept[b] (device int32 [m]).  Same order and error bits as tg_select_topk. */
+tg_status tg_select_topk_sweep(const float *scores, const uint8_t *doc_mask, int64_t n,
+                               const int32_t *ks, int32_t m, int32_t *kept_idx, int64_t stride,
+                               int32_t *n_kept, tg_stream stream);
+
+/* Random-K selection: keep k uniformly random document tokens (without replacement)
+ * and every question token, ascending -- the random-selector ablation of the
+ * TokenGate article ("How does TokenGate perform on benchmarks?": even random-K
+ * selection scores well on the co-adapted backbone).  Token i's random key is
+ * SplitMix64(seed, i) (Steele, Lea and Flood, 2014): x = seed + (i + 1) * 0x9E3779B97F4A7C15,
+ * x = (x ^ x >> 30) * 0xBF58476D1CE4E5B9, x = (x ^ x >> 27) * 0x94D049BB133111EB,
+ * x ^= x >> 31; the k document tokens with the largest (x >> 33) are kept, ties to the
+ * lower index.  Outputs and error bits as tg_select_topk. */
+tg_status tg_select_random_k(const uint8_t *doc_mask, int64_t n, int64_t k, uint64_t seed,
+                             int32_t *kept_idx, int64_t cap, int32_t *n_kept, tg_stream stream);
 
 /* --------------------------------------------------------------------------
  * tg_gather -- compaction of the kept tokens.

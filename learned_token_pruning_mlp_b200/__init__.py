@@ -21,6 +21,8 @@ from ._lib import (  # noqa: F401
     tg_gather,
     tg_get_device_error,
     tg_probe_wait_timeout,
+    tg_select_random_k,
     tg_select_topk,
+    tg_select_topk_sweep,
     tg_select_topk_varlen,
 )

@@ -46,6 +46,8 @@ _SIGNATURES = {
     "tg_gate_score": ([_vp, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp], ctypes.c_int),
     "tg_select_topk": ([_vp, _vp, _i64, _i64, _vp, _i64, _vp, _vp], ctypes.c_int),
     "tg_select_topk_varlen": ([_vp, _vp, _vp, _i32, _i64, _vp, _i64, _vp, _i64, _vp, _vp], ctypes.c_int),
+    "tg_select_topk_sweep": ([_vp, _vp, _i64, _vp, _i32, _vp, _i64, _vp, _vp], ctypes.c_int),
+    "tg_select_random_k": ([_vp, _i64, _i64, ctypes.c_uint64, _vp, _i64, _vp, _vp], ctypes.c_int),
     "tg_gather": ([_vp, _i64, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "tg_gated_attention": ([_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp, _vp], ctypes.c_int),
     "tg_gated_attention_varlen": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp, _vp],
@@ -151,6 +153,36 @@ def tg_select_topk_varlen(scores, doc_mask, cu_seqlens, k_per_seq, max_seqlen: i
         int(max_seqlen), _dev(kept_idx, torch.int32, "kept_idx"), int(cap), _dev(cu_kept, torch.int32, "cu_kept"),
         _stream(stream)))
     return kept_idx, cu_kept
+
+
+def tg_select_topk_sweep(scores, doc_mask, ks, kept_idx=None, n_kept=None, stride: Optional[int] = None,
+                         stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    n = scores.shape[0]
+    m = ks.numel()
+    stride = max(n, 1) if stride is None else stride
+    if kept_idx is None:
+        kept_idx = torch.empty(max(m * stride, 1), dtype=torch.int32, device=scores.device)
+    if n_kept is None:
+        n_kept = torch.empty(max(m, 1), dtype=torch.int32, device=scores.device)
+    _check("tg_select_topk_sweep", lib().tg_select_topk_sweep(
+        _dev(scores, torch.float32, "scores"), _dev(doc_mask, torch.uint8, "doc_mask"), n,
+        _dev(ks, torch.int32, "ks"), m, _dev(kept_idx, torch.int32, "kept_idx"), int(stride),
+        _dev(n_kept, torch.int32, "n_kept"), _stream(stream)))
+    return kept_idx, n_kept
+
+
+def tg_select_random_k(doc_mask, k: int, seed: int, kept_idx=None, n_kept=None, cap: Optional[int] = None,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    n = doc_mask.shape[0]
+    if kept_idx is None:
+        kept_idx = torch.empty(max(n, 1), dtype=torch.int32, device=doc_mask.device)
+    if n_kept is None:
+        n_kept = torch.empty(1, dtype=torch.int32, device=doc_mask.device)
+    cap = kept_idx.numel() if cap is None else cap
+    _check("tg_select_random_k", lib().tg_select_random_k(
+        _dev(doc_mask, torch.uint8, "doc_mask"), n, int(k), int(seed) & 0xFFFFFFFFFFFFFFFF,
+        _dev(kept_idx, torch.int32, "kept_idx"), int(cap), _dev(n_kept, torch.int32, "n_kept"), _stream(stream)))
+    return kept_idx, n_kept
 
 
 def tg_gather(hidden, kept_idx, n_rows: Optional[int] = None, n_kept=None, hidden_k=None, scores=None, s_k=None,

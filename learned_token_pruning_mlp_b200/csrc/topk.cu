@@ -136,34 +136,81 @@ __device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster,
   __syncthreads();
 }
 
-// One cluster per request.  Single-request mode: cu_seqlens == nullptr, the request is
-// [0, n_single) with budget k_single, base 0, and the CTA of rank 0 writes *n_kept.
-// Varlen mode: request b = cluster index, range from cu_seqlens, budget k_per_seq[b],
-// output offset cu_kept[b] (computed beforehand by seg_offsets_kernel).
+// Everything one launch of the cluster kernel needs (passed by value).
+struct TopkArgs {
+  const float *scores;        // nullptr in random mode
+  const uint8_t *mask;
+  int64_t n_single;           // single / sweep: the request is [0, n_single)
+  int64_t k_single;           // single: the budget
+  const int32_t *cu_seqlens;  // varlen: request b = [cu_seqlens[b], cu_seqlens[b+1])
+  const int32_t *k_per_seq;   // varlen: budgets
+  const int32_t *cu_kept;     // varlen: output offsets (from seg_offsets_kernel)
+  int64_t total;              // varlen: packed length
+  const int32_t *k_sweep;     // sweep: cluster b selects with budget k_sweep[b]
+  int64_t sweep_stride;       // sweep: cluster b writes kept_idx[b * stride ...]
+  int32_t *kept_idx;
+  int64_t cap;                // capacity per request (per budget in sweep mode)
+  int32_t *n_kept;            // single: [1]; sweep: [number of budgets]
+  uint64_t seed;              // random mode: key = SplitMix64(seed, position)
+  int random;
+  uint32_t *err;
+};
+
+// SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom number generators",
+// OOPSLA 2014): the state after n steps from ``seed`` is seed + n * golden gamma, and
+// the output mixes it with two multiply-xorshift rounds.  Counter-based, so any
+// position's value is computed directly.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t index) {
+  uint64_t z = seed + (index + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Random-mode order key of a document token: 31 random bits above every number key,
+// so the "largest" K keys are a uniformly random K-subset (ties by position).
+__device__ __forceinline__ uint32_t random_key(uint64_t seed, int64_t pos, bool doc) {
+  return doc ? (0x80000000u | static_cast<uint32_t>(splitmix64(seed, static_cast<uint64_t>(pos)) >> 33)) : 0u;
+}
+
+// One cluster per request.  Single-request mode: the request is [0, n_single) with
+// budget k_single, base 0, and the CTA of rank 0 writes *n_kept.  Varlen mode: request
+// b = cluster index, range from cu_seqlens, budget k_per_seq[b], output offset
+// cu_kept[b] (computed beforehand by seg_offsets_kernel).  Sweep mode: every cluster
+// selects from [0, n_single) with its own budget k_sweep[b] into its own output block.
 // kResident: every CTA's chunk fits one round (<= 16384 positions), keys stay in
 // registers; otherwise the keys are re-derived from the scores on every pass.
 template <bool kResident>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
-    topk_cluster_kernel(const float *__restrict__ scores, const uint8_t *__restrict__ mask, int64_t n_single,
-                        int64_t k_single, const int32_t *__restrict__ cu_seqlens, const int32_t *__restrict__ k_per_seq,
-                        const int32_t *__restrict__ cu_kept, int64_t total, int32_t *__restrict__ kept_idx,
-                        int64_t cap, int32_t *__restrict__ n_kept, uint32_t *err) {
+    topk_cluster_kernel(const TopkArgs args) {
   __shared__ TopkShared sh;
   tg::pdl_wait();
   tg::pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int seg = static_cast<int>(blockIdx.x) / kCluster;
+  const float *__restrict__ scores = args.scores;
+  const uint8_t *__restrict__ mask = args.mask;
+  const int32_t *__restrict__ cu_seqlens = args.cu_seqlens;
+  const int32_t *__restrict__ cu_kept = args.cu_kept;
+  int32_t *__restrict__ kept_idx = args.kept_idx;
+  uint32_t *err = args.err;
+  const int64_t cap = args.cap;
+  const int64_t total = args.total;
 
-  int64_t start = 0, end = n_single, k = k_single, base = 0;
+  int64_t start = 0, end = args.n_single, k = args.k_single, base = 0;
   if (cu_seqlens) {
     start = cu_seqlens[seg];
     end = cu_seqlens[seg + 1];
     start = start < 0 ? 0 : (start > total ? total : start);
     end = end < start ? start : (end > total ? total : end);
-    k = k_per_seq[seg];
+    k = args.k_per_seq[seg];
     base = cu_kept[seg];
+  } else if (args.k_sweep) {
+    k = args.k_sweep[seg];
+    base = static_cast<int64_t>(seg) * args.sweep_stride;
   }
+  const int64_t cap_end = args.k_sweep ? base + cap : cap;  // writes go below cap_end
   if (k < 0) k = 0;
   const int64_t len = end - start;
   // chunk: a multiple of kItems so that a thread's positions never straddle two CTAs
@@ -172,15 +219,25 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   const int64_t hi = lo + chunk < end ? lo + chunk : end;
   const int m = lo < hi ? static_cast<int>(hi - lo) : 0;
   const int rounds = kResident ? 1 : (m + kRound - 1) / kRound;
+  // the launcher picks the register-resident variant from the caller's length bound; a
+  // request longer than that bound cannot be handled by it and is reported
+  if (kResident && m > kRound && threadIdx.x == 0) tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
 
   // 16-byte vector loads when this CTA's chunk starts aligned (always for a single request
   // with aligned buffers; varlen requests may start anywhere and then use scalar loads)
-  const bool vec = ((reinterpret_cast<uintptr_t>(scores + lo) | reinterpret_cast<uintptr_t>(mask + lo)) & 15u) == 0;
+  const bool vec = !args.random &&
+                   ((reinterpret_cast<uintptr_t>(scores + lo) | reinterpret_cast<uintptr_t>(mask + lo)) & 15u) == 0;
   uint32_t keys[kItems];
   // positions past the chunk get key 0 and are excluded from every count by valid()
   auto load_keys = [&](int round) {
     const int i0 = round * kRound + threadIdx.x * kItems;
-    if (vec && i0 + kItems <= m) {
+    if (args.random) {
+#pragma unroll
+      for (int e = 0; e < kItems; ++e) {
+        const int i = i0 + e;
+        keys[e] = i < m ? random_key(args.seed, lo + i, mask[lo + i] != 0) : 0u;
+      }
+    } else if (vec && i0 + kItems <= m) {
       float f[kItems];
       const float4 *s4 = reinterpret_cast<const float4 *>(scores + lo + i0);
 #pragma unroll
@@ -326,7 +383,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       sh.bcast[1] = base + keep_incl - keep;
     }
     if (lane == 0) {
-      if (!cu_seqlens && rank == 0) *n_kept = static_cast<int32_t>(nt);
+      if (!cu_seqlens && rank == 0) args.n_kept[args.k_sweep ? seg : 0] = static_cast<int32_t>(nt);
       if (cu_seqlens && rank == 0 && static_cast<long long>(cu_kept[seg + 1]) - base != nt)
         tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
     }
@@ -362,7 +419,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     while (bits) {
       const int e = __ffs(bits) - 1;
       bits &= bits - 1;
-      if (pos < cap) {
+      if (pos < cap_end) {
         kept_idx[pos] = static_cast<int32_t>(p0 + e);
       } else {
         tg::set_device_error(err, TG_DEVERR_CAPACITY);
@@ -417,15 +474,9 @@ __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__rest
   }
 }
 
-cudaError_t launch_cluster(bool resident, unsigned grid, cudaStream_t s, const float *scores, const uint8_t *mask,
-                           int64_t n_single, int64_t k_single, const int32_t *cu, const int32_t *kps,
-                           const int32_t *cu_kept, int64_t total, int32_t *kept_idx, int64_t cap, int32_t *n_kept,
-                           uint32_t *err) {
-  if (resident)
-    return tg::launch_pdl(topk_cluster_kernel<true>, dim3(grid), dim3(kThreads), 0, s, scores, mask, n_single, k_single,
-                          cu, kps, cu_kept, total, kept_idx, cap, n_kept, err);
-  return tg::launch_pdl(topk_cluster_kernel<false>, dim3(grid), dim3(kThreads), 0, s, scores, mask, n_single, k_single,
-                        cu, kps, cu_kept, total, kept_idx, cap, n_kept, err);
+cudaError_t launch_cluster(bool resident, unsigned grid, cudaStream_t s, const TopkArgs &a) {
+  if (resident) return tg::launch_pdl(topk_cluster_kernel<true>, dim3(grid), dim3(kThreads), 0, s, a);
+  return tg::launch_pdl(topk_cluster_kernel<false>, dim3(grid), dim3(kThreads), 0, s, a);
 }
 
 // chunk per CTA for a request of ``len`` positions (as the kernel computes it)
@@ -444,8 +495,75 @@ extern "C" tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask
   if (cap > 0 && !kept_idx) return tg::fail(TG_ERR_INVALID_ARG, "kept_idx is NULL");
   uint32_t *err = tg::device_error_word();
   if (!err) return TG_ERR_CUDA;
-  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), scores,
-                                      doc_mask, n, k, nullptr, nullptr, nullptr, n, kept_idx, cap, n_kept, err);
+  TopkArgs a = {};
+  a.scores = scores;
+  a.mask = doc_mask;
+  a.n_single = n;
+  a.k_single = k;
+  a.total = n;
+  a.kept_idx = kept_idx;
+  a.cap = cap;
+  a.n_kept = n_kept;
+  a.err = err;
+  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
+  return tg::check_launch("topk_cluster_kernel");
+}
+
+extern "C" tg_status tg_select_random_k(const uint8_t *doc_mask, int64_t n, int64_t k, uint64_t seed,
+                                        int32_t *kept_idx, int64_t cap, int32_t *n_kept, tg_stream stream) {
+  tg::clear_detail();
+  if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
+  if (k < 0) return tg::fail(TG_ERR_INVALID_ARG, "k must be >= 0");
+  if (cap < 0) return tg::fail(TG_ERR_INVALID_ARG, "cap must be >= 0");
+  if (!n_kept) return tg::fail(TG_ERR_INVALID_ARG, "n_kept is NULL");
+  if (n > 0 && !doc_mask) return tg::fail(TG_ERR_INVALID_ARG, "doc_mask is NULL");
+  if (cap > 0 && !kept_idx) return tg::fail(TG_ERR_INVALID_ARG, "kept_idx is NULL");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  TopkArgs a = {};
+  a.mask = doc_mask;
+  a.n_single = n;
+  a.k_single = k;
+  a.total = n;
+  a.kept_idx = kept_idx;
+  a.cap = cap;
+  a.n_kept = n_kept;
+  a.seed = seed;
+  a.random = 1;
+  a.err = err;
+  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
+  return tg::check_launch("topk_cluster_kernel");
+}
+
+extern "C" tg_status tg_select_topk_sweep(const float *scores, const uint8_t *doc_mask, int64_t n,
+                                          const int32_t *ks, int32_t m, int32_t *kept_idx, int64_t stride,
+                                          int32_t *n_kept, tg_stream stream) {
+  tg::clear_detail();
+  if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
+  if (m < 0 || m > 65535) return tg::fail(TG_ERR_INVALID_ARG, "the number of budgets must be in [0, 65535]");
+  if (stride < 0 || (m > 0 && stride > 0x7FFFFFFFLL / m))
+    return tg::fail(TG_ERR_INVALID_ARG, "stride must be >= 0 and m * stride < 2^31");
+  if (m == 0) return TG_OK;
+  if (!ks || !n_kept) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (n > 0 && (!scores || !doc_mask)) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (stride > 0 && !kept_idx) return tg::fail(TG_ERR_INVALID_ARG, "kept_idx is NULL");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  TopkArgs a = {};
+  a.scores = scores;
+  a.mask = doc_mask;
+  a.n_single = n;
+  a.total = n;
+  a.k_sweep = ks;
+  a.sweep_stride = stride;
+  a.kept_idx = kept_idx;
+  a.cap = stride;
+  a.n_kept = n_kept;
+  a.err = err;
+  const cudaError_t e =
+      launch_cluster(chunk_of(n) <= kRound, static_cast<unsigned>(m) * kCluster, static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
@@ -470,10 +588,19 @@ extern "C" tg_status tg_select_topk_varlen(const float *scores, const uint8_t *d
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "seg_offsets_kernel launch: %s", cudaGetErrorString(e));
   tg_status st = tg::check_launch("seg_offsets_kernel");
   if (st != TG_OK || B == 0) return st;
-  // the resident variant is only chosen when every request's chunk fits; a request longer
-  // than max_seqlen would need the other variant, so max_seqlen must bound them all
-  e = launch_cluster(chunk_of(max_seqlen) <= kRound, static_cast<unsigned>(B) * kCluster, s, scores, doc_mask, 0, 0,
-                     cu_seqlens, k_per_seq, cu_kept, total, kept_idx, cap, nullptr, err);
+  TopkArgs a = {};
+  a.scores = scores;
+  a.mask = doc_mask;
+  a.cu_seqlens = cu_seqlens;
+  a.k_per_seq = k_per_seq;
+  a.cu_kept = cu_kept;
+  a.total = total;
+  a.kept_idx = kept_idx;
+  a.cap = cap;
+  a.err = err;
+  // the register-resident variant is chosen when max_seqlen fits it; a request longer
+  // than max_seqlen then sets TG_DEVERR_BAD_SEQLENS
+  e = launch_cluster(chunk_of(max_seqlen) <= kRound, static_cast<unsigned>(B) * kCluster, s, a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }

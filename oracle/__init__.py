@@ -41,6 +41,10 @@ def lib():
         L.orc_gather.restype = None
         L.orc_gated_attention_rows.argtypes = [vp, vp, vp, vp, vp, f64, i64, i32, i32, i32, vp, i64, vp]
         L.orc_gated_attention_rows.restype = None
+        L.orc_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        L.orc_splitmix64.restype = ctypes.c_uint64
+        L.orc_select_random_k.argtypes = [vp, i64, i64, ctypes.c_uint64, vp]
+        L.orc_select_random_k.restype = i64
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
@@ -102,6 +106,25 @@ def select_topk_varlen(scores, doc_mask, cu_seqlens: Sequence[int], ks: Sequence
         cu_kept.append(cu_kept[-1] + len(kept))
     kept_all = np.concatenate(parts) if parts else np.zeros(0, np.int32)
     return kept_all, np.asarray(cu_kept, dtype=np.int32)
+
+
+def select_topk_sweep(scores, doc_mask, ks: Sequence[int]):
+    """The selection at every budget of ``ks``: a list of kept-index arrays."""
+    return [select_topk(scores, doc_mask, int(k)) for k in ks]
+
+
+def splitmix64(seed: int, index: int) -> int:
+    """The (index + 1)-th output of SplitMix64 seeded with ``seed``."""
+    return int(lib().orc_splitmix64(seed & 0xFFFFFFFFFFFFFFFF, index))
+
+
+def select_random_k(doc_mask, k: int, seed: int) -> np.ndarray:
+    """k uniformly random document tokens (SplitMix64 keys, ties to the lower index) plus
+    every question token, ascending int32."""
+    m = _np(doc_mask, np.uint8)
+    out = np.empty(max(len(m), 1), dtype=np.int32)
+    cnt = lib().orc_select_random_k(_ptr(m), len(m), int(k), seed & 0xFFFFFFFFFFFFFFFF, _ptr(out))
+    return out[:cnt].copy()
 
 
 # --------------------------------------------------------------------------- gather

@@ -143,6 +143,64 @@ int64_t orc_select_topk(const float *scores, const uint8_t *doc_mask, int64_t n,
 }
 
 /* ------------------------------------------------------------------------ *
+ * Random-K selection (the random-selector ablation of the TokenGate article,
+ * "How does TokenGate perform on benchmarks?").  Each document token draws a
+ * random key from SplitMix64 (Steele, Lea and Flood, "Fast splittable
+ * pseudorandom number generators", OOPSLA 2014) as a counter-based generator:
+ * the value for position i is the (i + 1)-th output of the generator seeded with
+ * ``seed``.  The k document tokens with the largest key >> 33 are kept (ties to
+ * the lower index), every question token is kept, output ascending.
+ * ------------------------------------------------------------------------ */
+uint64_t orc_splitmix64(uint64_t seed, uint64_t index)
+{
+    uint64_t x = seed;
+    /* advance the state index + 1 times by the golden gamma, then mix */
+    x += (index + 1) * 0x9E3779B97F4A7C15ull;
+    uint64_t z = x;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+typedef struct {
+    uint64_t key;
+    int32_t i;
+} keyed_index;
+
+static int cmp_key_desc(const void *pa, const void *pb)
+{
+    const keyed_index *a = (const keyed_index *)pa, *b = (const keyed_index *)pb;
+    if (a->key != b->key) return a->key > b->key ? -1 : 1;
+    return a->i < b->i ? -1 : (a->i > b->i);
+}
+
+int64_t orc_select_random_k(const uint8_t *doc_mask, int64_t n, int64_t k, uint64_t seed, int32_t *kept)
+{
+    int64_t n_doc = 0;
+    for (int64_t i = 0; i < n; ++i) n_doc += doc_mask[i] != 0;
+    keyed_index *doc = (keyed_index *)malloc(sizeof(keyed_index) * (size_t)(n_doc > 0 ? n_doc : 1));
+    int64_t t = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (doc_mask[i]) {
+            doc[t].key = orc_splitmix64(seed, (uint64_t)i) >> 33;
+            doc[t].i = (int32_t)i;
+            ++t;
+        }
+    qsort(doc, (size_t)n_doc, sizeof(keyed_index), cmp_key_desc);
+    const int64_t take = k < 0 ? 0 : (k < n_doc ? k : n_doc);
+    uint8_t *keep = (uint8_t *)calloc((size_t)(n > 0 ? n : 1), 1);
+    for (int64_t r = 0; r < take; ++r) keep[doc[r].i] = 1;
+    for (int64_t i = 0; i < n; ++i)
+        if (!doc_mask[i]) keep[i] = 1;
+    int64_t m = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (keep[i]) kept[m++] = (int32_t)i;
+    free(keep);
+    free(doc);
+    return m;
+}
+
+/* ------------------------------------------------------------------------ *
  * Gather / compaction.
  * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
  * forward): layers above L process only the kept tokens.

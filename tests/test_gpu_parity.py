@@ -173,6 +173,38 @@ def test_topk_varlen_bit_exact(lens):
     assert bits & ~tg.TG_DEVERR_K_GT_NDOC == 0
 
 
+@pytest.mark.parametrize("n", [1, 100, 4097, 131072, 200003])
+def test_random_k_bit_exact(n):
+    rng = np.random.default_rng(n + 7)
+    mask = (rng.random(n) < 0.9).astype(np.uint8)
+    n_doc = int(mask.sum())
+    for seed in (0, 12345, 2**64 - 1):
+        for k in sorted({0, 1, n_doc // 3, n_doc, n_doc + 5}):
+            kept, nk = tg.tg_select_random_k(torch.as_tensor(mask).to(DEV), k, seed)
+            cnt = int(nk.item())
+            ref = oracle.select_random_k(mask, k, seed)
+            assert cnt == len(ref)
+            assert np.array_equal(kept[:cnt].cpu().numpy(), ref), (n, seed, k)
+    tg.tg_get_device_error()  # budgets above the document set TG_DEVERR_K_GT_NDOC
+
+
+@pytest.mark.parametrize("n", [777, 131072])
+def test_topk_sweep_bit_exact(n):
+    s = W.mixture_scores(n, n).numpy()
+    mask = np.ones(n, np.uint8)
+    mask[-(n // 16):] = 0
+    n_doc = int(mask.sum())
+    ks = [0, 1, 64, n_doc // 2, n_doc, n_doc + 9]
+    kept, nk = tg.tg_select_topk_sweep(torch.as_tensor(s).to(DEV), torch.as_tensor(mask).to(DEV),
+                                       torch.tensor(ks, dtype=torch.int32).to(DEV), stride=n)
+    nk = nk.cpu().numpy()
+    kept = kept.cpu().numpy()
+    for b, ref in enumerate(oracle.select_topk_sweep(s, mask, ks)):
+        assert nk[b] == len(ref)
+        assert np.array_equal(kept[b * n:b * n + len(ref)], ref), ks[b]
+    tg.tg_get_device_error()
+
+
 # =============================================================================== gate
 @pytest.mark.parametrize("n,d,h", [(512, 256, 64), (1000, 2048, 256), (300, 200, 48), (129, 64, 16), (16384, 2048, 256)])
 def test_gate_scores_within_tolerance(n, d, h):

@@ -383,3 +383,46 @@ def test_pruned_tokens_never_influence_outputs():
     for a, b in zip(clean, poisoned):
         assert np.array_equal(a, b)
         assert not np.isnan(np.asarray(b, dtype=np.float64)).any()
+
+
+# ============================================================================ random-K and sweep
+def test_splitmix64_matches_published_outputs():
+    with open(os.path.join(GOLDEN, "splitmix64_vectors.json")) as f:
+        g = json.load(f)
+    got = [oracle.splitmix64(g["seed"], i) for i in range(len(g["outputs"]))]
+    assert got == [int(v) for v in g["outputs"]]
+
+
+def test_random_k_is_top_k_of_the_random_keys():
+    rng = np.random.default_rng(4)
+    for n in (1, 37, 500):
+        m = (rng.random(n) < 0.75).astype(np.uint8)
+        for seed in (0, 7, 2**63 + 5):
+            keys = np.asarray([oracle.splitmix64(seed, i) >> 33 for i in range(n)], dtype=np.float64)
+            for k in (0, 1, int(m.sum()) // 2, int(m.sum()), int(m.sum()) + 3):
+                got = oracle.select_random_k(m, k, seed)
+                assert got.tolist() == _brute_topk(keys, m, k).tolist()
+
+
+def test_random_k_is_roughly_uniform():
+    # every document position is kept with probability k / n_doc over seeds
+    n, k, trials = 64, 16, 400
+    m = np.ones(n, dtype=np.uint8)
+    hits = np.zeros(n)
+    for seed in range(trials):
+        hits[oracle.select_random_k(m, k, seed)] += 1
+    freq = hits / trials
+    assert abs(freq.mean() - k / n) < 1e-12
+    assert np.all(np.abs(freq - k / n) < 0.12)
+
+
+def test_sweep_is_nested_and_matches_single_budgets():
+    s = W.mixture_scores(3000, 9).numpy()
+    m = np.ones(3000, dtype=np.uint8)
+    m[-100:] = 0
+    ks = [0, 10, 500, 2900, 5000]
+    sets = oracle.select_topk_sweep(s, m, ks)
+    for k, kept in zip(ks, sets):
+        assert kept.tolist() == oracle.select_topk(s, m, k).tolist()
+    for a, b in zip(sets, sets[1:]):
+        assert set(a.tolist()) <= set(b.tolist())
