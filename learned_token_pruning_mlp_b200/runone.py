@@ -3,6 +3,8 @@
     python -m learned_token_pruning_mlp_b200.runone attention --S 8704 --repeat 3
     python -m learned_token_pruning_mlp_b200.runone gate --n 131072
     python -m learned_token_pruning_mlp_b200.runone topk --n 131072 --k 8192
+    python -m learned_token_pruning_mlp_b200.runone randomk --n 131072 --k 8192
+    python -m learned_token_pruning_mlp_b200.runone sweep --n 131072 --k 8192   # budgets k/4, k/2, k, 2k
     python -m learned_token_pruning_mlp_b200.runone gather --n 131072 --rows 8704
 
 Each call is timed with CUDA events on the launching stream (after one warm-up
@@ -23,7 +25,7 @@ from . import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("call", choices=["gate", "topk", "gather", "attention"])
+    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention"])
     ap.add_argument("--n", type=int, default=131072)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--h", type=int, default=256)
@@ -56,6 +58,20 @@ def main():
         kept = torch.empty(a.n, dtype=torch.int32, device=dev)
         nk = torch.empty(1, dtype=torch.int32, device=dev)
         fn = lambda: tg.tg_select_topk(s, m, a.k, kept_idx=kept, n_kept=nk)
+    elif a.call == "randomk":
+        m = torch.ones(a.n, dtype=torch.uint8, device=dev)
+        m[-512:] = 0
+        kept = torch.empty(a.n, dtype=torch.int32, device=dev)
+        nk = torch.empty(1, dtype=torch.int32, device=dev)
+        fn = lambda: tg.tg_select_random_k(m, a.k, 42, kept_idx=kept, n_kept=nk)
+    elif a.call == "sweep":
+        s = W.mixture_scores(a.n, 3).to(dev)
+        m = torch.ones(a.n, dtype=torch.uint8, device=dev)
+        m[-512:] = 0
+        ks = torch.tensor([a.k // 4, a.k // 2, a.k, 2 * a.k], dtype=torch.int32, device=dev)
+        kept = torch.empty(4 * a.n, dtype=torch.int32, device=dev)
+        nk = torch.empty(4, dtype=torch.int32, device=dev)
+        fn = lambda: tg.tg_select_topk_sweep(s, m, ks, kept_idx=kept, n_kept=nk, stride=a.n)
     elif a.call == "gather":
         hidden = torch.randn(a.n, a.d, generator=g).to(torch.bfloat16).to(dev)
         sc = torch.randn(a.n, generator=g).to(dev)
