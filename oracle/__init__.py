@@ -11,8 +11,8 @@ Two independent implementations live here:
 
 Source: the MarkTechPost TokenGate article, sections "How does TokenGate
 learned token pruning work?" (gate, top-K, question never pruned, pruned
-forward) and "What is token-gated attention?" (score as logit bias, per-head
-gain, temperature).  Each function below restates the definition it follows.
+forward, kept tokens at their prompt positions) and "What is token-gated
+attention?" (score as logit bias, per-head gain, temperature).  Each function below restates the definition it follows.
 """
 from __future__ import annotations
 
@@ -45,6 +45,10 @@ def lib():
         L.orc_splitmix64.restype = ctypes.c_uint64
         L.orc_select_random_k.argtypes = [vp, i64, i64, ctypes.c_uint64, vp]
         L.orc_select_random_k.restype = i64
+        L.orc_qkv_rope_rows.argtypes = [vp, i32, vp, vp, f64, i32, i32, i32, vp, vp, f64, vp, i64, vp, vp, vp]
+        L.orc_qkv_rope_rows.restype = None
+        L.orc_linear_rows.argtypes = [vp, i32, vp, i32, vp, vp, i64, vp]
+        L.orc_linear_rows.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
@@ -176,6 +180,40 @@ def gated_attention_varlen(Q, K, V, s, gain, tau: float, cu_seqlens: Sequence[in
         out[sel] = gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], _np(s, np.float32)[lo:hi], gain, tau,
                                    rows=rows_all[sel] - lo)
     return out
+
+
+# --------------------------------------------------------------------------- projections
+def qkv_rope(hidden, W_qkv, positions, base: float, Hq: int, Hkv: int, D: int, q_norm=None, k_norm=None,
+             eps: float = 1e-6, rows: Optional[Sequence[int]] = None):
+    """[Q K V] = W_qkv x_i; optional per-head RMS norm of Q / K heads; rotary embedding of Q / K heads
+    at ``positions[i]`` with pairs (j, j + D/2) and angles p * base^(-2j/D).
+    Returns fp64 (Q [R, Hq, D], K [R, Hkv, D], V [R, Hkv, D]) for the listed rows (all when None)."""
+    S, d = hidden.shape
+    hb, wb = _bf16_bits(hidden), _bf16_bits(W_qkv)
+    assert wb.shape == ((Hq + 2 * Hkv) * D, d)
+    pv = _np(positions, np.int32)
+    qn = _bf16_bits(q_norm) if q_norm is not None else None
+    kn = _bf16_bits(k_norm) if k_norm is not None else None
+    r = np.arange(S, dtype=np.int64) if rows is None else _np(rows, np.int64)
+    Q = np.empty((len(r), Hq, D))
+    K = np.empty((len(r), Hkv, D))
+    V = np.empty((len(r), Hkv, D))
+    lib().orc_qkv_rope_rows(_ptr(hb), d, _ptr(wb), _ptr(pv), float(base), Hq, Hkv, D,
+                            _ptr(qn) if qn is not None else None, _ptr(kn) if kn is not None else None,
+                            float(eps), _ptr(r), len(r), _ptr(Q), _ptr(K), _ptr(V))
+    return Q, K, V
+
+
+def linear(x, W, residual=None, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """y_i = W x_i (+ residual_i) in fp64 over the bf16 inputs; fp64 [len(rows), N]."""
+    M, K = x.shape
+    N = W.shape[0]
+    xb, wb = _bf16_bits(x), _bf16_bits(W)
+    rb = _bf16_bits(residual) if residual is not None else None
+    r = np.arange(M, dtype=np.int64) if rows is None else _np(rows, np.int64)
+    y = np.empty((len(r), N))
+    lib().orc_linear_rows(_ptr(xb), K, _ptr(wb), N, _ptr(rb) if rb is not None else None, _ptr(r), len(r), _ptr(y))
+    return y
 
 
 def sampled_rows(S: int, seed: int, head: int = 128, tail: int = 128, rand: int = 256) -> np.ndarray:

@@ -26,6 +26,10 @@
  *                 additive key bias), row 0 = V[0], bias-shift invariance,
  *                 duplicated-KV-head equivalence, convex-hull bound,
  *                 pruned keys never influence an output.
+ *   projections -- torch fp64 matmul (positions 0, no norm), a hand-worked
+ *                 rotary fixture, relative-position invariance of q.k, norm
+ *                 preservation, scale invariance of the per-head norm, and
+ *                 pruning commuting with projection at original positions.
  */
 #include <math.h>
 #include <stdint.h>
@@ -278,6 +282,104 @@ void orc_gated_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16
         }
         free(q);
         free(l);
+    }
+}
+
+/* ------------------------------------------------------------------------ *
+ * Projections of a pruned layer (the layers above the gate).
+ * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
+ * forward): the layers above L run on the kept tokens only, and those tokens
+ * stay at their prompt positions.  The article names the Qwen3 backbones but no
+ * layer formula; the plainest reading of a Qwen3 attention block is taken:
+ *
+ *   y      = W_qkv x_i                   W_qkv: bf16 [(Hq + 2 Hkv) D, d], rows =
+ *                                        Q heads, then K heads, then V heads
+ *   per Q / K head (optional, Qwen3 style, weight w of length D):
+ *          u_c = y_c / sqrt(mean_c(y_c^2) + eps) * w_c
+ *   rotary embedding of Q / K heads at position p_i, pairs (j, j + D/2):
+ *          phi_j = p_i * base^(-2j / D)                 (j < D/2)
+ *          out_j       = u_j cos phi_j - u_{j+D/2} sin phi_j
+ *          out_{j+D/2} = u_{j+D/2} cos phi_j + u_j sin phi_j
+ *   V heads are neither normalised nor rotated.
+ *
+ * hidden: bf16 [S, d]; positions: int32 [S] (the original token index of every
+ * kept row); q_norm / k_norm: bf16 [D] or NULL (no normalisation).  Only the
+ * listed rows are computed; Q: double [n_rows, Hq, D], K and V: double
+ * [n_rows, Hkv, D].
+ * ------------------------------------------------------------------------ */
+static void rms_normalise(double *u, int32_t D, const uint16_t *w, double eps)
+{
+    double ss = 0.0;
+    for (int32_t c = 0; c < D; ++c) ss += u[c] * u[c];
+    const double r = 1.0 / sqrt(ss / (double)D + eps);
+    for (int32_t c = 0; c < D; ++c) u[c] = u[c] * r * bf16_value(w[c]);
+}
+
+static void rotate(const double *u, int32_t D, int64_t pos, double base, double *out)
+{
+    const int32_t half = D / 2;
+    for (int32_t j = 0; j < half; ++j) {
+        const double phi = (double)pos * pow(base, -2.0 * (double)j / (double)D);
+        const double c = cos(phi), s = sin(phi);
+        out[j] = u[j] * c - u[j + half] * s;
+        out[j + half] = u[j + half] * c + u[j] * s;
+    }
+}
+
+void orc_qkv_rope_rows(const uint16_t *hidden, int32_t d, const uint16_t *W_qkv,
+                       const int32_t *positions, double base, int32_t Hq, int32_t Hkv,
+                       int32_t D, const uint16_t *q_norm, const uint16_t *k_norm, double eps,
+                       const int64_t *rows, int64_t n_rows, double *Q, double *K, double *V)
+{
+    const int32_t n_out = (Hq + 2 * Hkv) * D;
+#pragma omp parallel
+    {
+        double *y = (double *)malloc(sizeof(double) * (size_t)n_out);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            const int64_t i = rows[r];
+            const uint16_t *x = hidden + (size_t)i * (size_t)d;
+            for (int32_t o = 0; o < n_out; ++o) {
+                const uint16_t *w = W_qkv + (size_t)o * (size_t)d;
+                double acc = 0.0;
+                for (int32_t k = 0; k < d; ++k) acc += bf16_value(w[k]) * bf16_value(x[k]);
+                y[o] = acc;
+            }
+            for (int32_t hh = 0; hh < Hq + Hkv; ++hh) {
+                double *u = y + (size_t)hh * D;
+                const int is_q = hh < Hq;
+                const uint16_t *nw = is_q ? q_norm : k_norm;
+                if (nw) rms_normalise(u, D, nw, eps);
+                double *dst = is_q ? Q + ((size_t)r * Hq + hh) * D
+                                   : K + ((size_t)r * Hkv + (hh - Hq)) * D;
+                rotate(u, D, positions[i], base, dst);
+            }
+            for (int32_t g = 0; g < Hkv; ++g)
+                memcpy(V + ((size_t)r * Hkv + g) * D, y + (size_t)(Hq + Hkv + g) * D,
+                       sizeof(double) * (size_t)D);
+        }
+        free(y);
+    }
+}
+
+/* Output projection (o_proj) with an optional residual add:
+ *     y_i = W x_i (+ residual_i)
+ * x: bf16 [M, K]; W: bf16 [N, K] (nn.Linear layout); residual: bf16 [M, N] or
+ * NULL.  Only the listed rows are computed; y: double [n_rows, N]. */
+void orc_linear_rows(const uint16_t *x, int32_t K, const uint16_t *W, int32_t N,
+                     const uint16_t *residual, const int64_t *rows, int64_t n_rows, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t i = rows[r];
+        const uint16_t *xi = x + (size_t)i * (size_t)K;
+        for (int32_t o = 0; o < N; ++o) {
+            const uint16_t *w = W + (size_t)o * (size_t)K;
+            double acc = 0.0;
+            for (int32_t k = 0; k < K; ++k) acc += bf16_value(w[k]) * bf16_value(xi[k]);
+            if (residual) acc += bf16_value(residual[(size_t)i * (size_t)N + o]);
+            y[(size_t)r * N + o] = acc;
+        }
     }
 }
 

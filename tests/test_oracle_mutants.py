@@ -96,3 +96,77 @@ def test_gate_pin_rejects_wrong_activation_and_transposed_weight():
     for bad in (relu, transposed, no_b1):
         assert _rejected(bad, ref)
     np.testing.assert_allclose(twin.gate_score(hidden, W1, b1, W2, b2), ref, rtol=1e-12, atol=1e-12)
+
+
+def _qkv_rope_variant(x, Wt, positions, base, Hq, Hkv, D, q_norm=None, k_norm=None, eps=1e-6, *,
+                      pairs="half", sign=1.0, expo=2.0, norm_scope="head", use_rows=False):
+    """A numpy copy of the projection + per-head norm + rotary definition with one planted mistake."""
+    y = x.double().numpy() @ Wt.double().numpy().T
+    S = y.shape[0]
+    pos = np.arange(S) if use_rows else np.asarray(positions, np.float64)
+    out = []
+    for lo, H, w in ((0, Hq, q_norm), (Hq * D, Hkv, k_norm)):
+        u = y[:, lo:lo + H * D].reshape(S, H, D).copy()
+        if w is not None:
+            wv = w.double().numpy()
+            if norm_scope == "head":
+                ms = np.mean(u ** 2, axis=-1, keepdims=True)
+            else:
+                ms = np.mean(u.reshape(S, -1) ** 2, axis=-1)[:, None, None]
+            u = u / np.sqrt(ms + eps) * wv
+        j = np.arange(D // 2)
+        phi = pos[:, None] * base ** (-expo * j / D)
+        c, s = np.cos(phi)[:, None, :], np.sin(phi)[:, None, :]
+        if pairs == "half":
+            a, b = u[..., :D // 2], u[..., D // 2:]
+        else:
+            a, b = u[..., 0::2], u[..., 1::2]
+        ra, rb = a * c - sign * b * s, b * c + sign * a * s
+        r = np.empty_like(u)
+        if pairs == "half":
+            r[..., :D // 2], r[..., D // 2:] = ra, rb
+        else:
+            r[..., 0::2], r[..., 1::2] = ra, rb
+        out.append(r)
+    v = y[:, (Hq + Hkv) * D:].reshape(S, Hkv, D)
+    return out[0], out[1], v
+
+
+def test_projection_pins_reject_planted_mistakes():
+    from test_oracle_pins import _load_rope_golden, _rope_golden_case, _proj_case
+    g = _load_rope_golden()
+
+    def golden_ok(**mut):
+        fn = lambda *a, **k: _qkv_rope_variant(*a, **k, **mut)  # noqa: E731
+        for c in g["cases"]:
+            Q, K, V = _rope_golden_case(fn, g, c)
+            if not np.allclose(Q[0, 0], c["q"], rtol=0, atol=g["tol"]):
+                return False
+        return True
+
+    assert golden_ok()                         # the unmutated copy passes
+    assert not golden_ok(pairs="interleaved")  # (2j, 2j+1) pairs instead of (j, j + D/2)
+    assert not golden_ok(sign=-1.0)            # rotation the wrong way
+    assert not golden_ok(expo=1.0)             # base^(-j/D) instead of base^(-2j/D)
+
+    # norm over all heads of a row instead of per head: the per-head unit-RMS pin fails
+    Hq, Hkv, D = 4, 2, 32
+    x, Wq, _, _ = _proj_case(8, Hq, Hkv, D, 64, 51)
+    ones = _bf16_ones(D)
+    pos = np.arange(8) * 3
+    Q, _, _ = _qkv_rope_variant(x, Wq, pos, 1e6, Hq, Hkv, D, ones, ones, 0.0)
+    assert np.allclose(np.mean(Q ** 2, axis=-1), 1.0, rtol=1e-12)
+    Qm, _, _ = _qkv_rope_variant(x, Wq, pos, 1e6, Hq, Hkv, D, ones, ones, 0.0, norm_scope="row")
+    assert not np.allclose(np.mean(Qm ** 2, axis=-1), 1.0, rtol=1e-6)
+
+    # compacted row numbers as positions: pruning no longer commutes with the projection
+    x, Wq, qn, kn = _proj_case(64, 2, 1, 32, 64, 61)
+    kept = np.sort(np.random.default_rng(1).choice(64, 20, replace=False))
+    full = _qkv_rope_variant(x, Wq, np.arange(64), 1e6, 2, 1, 32, qn, kn)
+    sub = x[torch.as_tensor(kept)]
+    assert np.allclose(full[0][kept], _qkv_rope_variant(sub, Wq, kept, 1e6, 2, 1, 32, qn, kn)[0])
+    assert not np.allclose(full[0][kept], _qkv_rope_variant(sub, Wq, kept, 1e6, 2, 1, 32, qn, kn, use_rows=True)[0])
+
+
+def _bf16_ones(D):
+    return torch.ones(D, dtype=torch.bfloat16)

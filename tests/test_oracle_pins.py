@@ -426,3 +426,115 @@ def test_sweep_is_nested_and_matches_single_budgets():
         assert kept.tolist() == oracle.select_topk(s, m, k).tolist()
     for a, b in zip(sets, sets[1:]):
         assert set(a.tolist()) <= set(b.tolist())
+
+
+# ============================================================================ projections
+def test_linear_matches_torch_fp64_with_and_without_residual():
+    x = _rand_bf16((37, 72), 11)
+    Wt = _rand_bf16((96, 72), 12, 0.1)
+    res = _rand_bf16((37, 96), 13)
+    ref = F.linear(x.double(), Wt.double()).numpy()
+    assert np.allclose(oracle.linear(x, Wt), ref, rtol=1e-13, atol=1e-13)
+    assert np.allclose(oracle.linear(x, Wt, res), ref + res.double().numpy(), rtol=1e-13, atol=1e-13)
+    rows = [36, 0, 5]
+    assert np.array_equal(oracle.linear(x, Wt, res, rows=rows), oracle.linear(x, Wt, res)[rows])
+
+
+def test_qkv_at_position_zero_without_norm_is_the_plain_projection():
+    Hq, Hkv, D, d = 4, 2, 16, 48
+    x = _rand_bf16((9, d), 21)
+    Wq = _rand_bf16(((Hq + 2 * Hkv) * D, d), 22, 0.2)
+    Q, K, V = oracle.qkv_rope(x, Wq, np.zeros(9, np.int32), 1e6, Hq, Hkv, D)
+    y = F.linear(x.double(), Wq.double()).numpy()
+    assert np.allclose(Q.reshape(9, -1), y[:, :Hq * D], rtol=1e-13, atol=1e-13)
+    assert np.allclose(K.reshape(9, -1), y[:, Hq * D:(Hq + Hkv) * D], rtol=1e-13, atol=1e-13)
+    assert np.allclose(V.reshape(9, -1), y[:, (Hq + Hkv) * D:], rtol=1e-13, atol=1e-13)
+
+
+def _load_rope_golden():
+    with open(os.path.join(GOLDEN, "rope_worked.json")) as f:
+        return json.load(f)
+
+
+def _rope_golden_case(fn, g, c):
+    """Run ``fn`` (an oracle-shaped qkv_rope) on one fixture case: W_qkv = three 4x4 identities."""
+    D = g["D"]
+    Wt = _bf16(np.vstack([np.eye(D)] * 3))
+    x = _bf16(np.asarray(c["x"], np.float32)[None, :])
+    w = _bf16(np.ones(D, np.float32)) if c["norm"] else None
+    return fn(x, Wt, np.asarray([c["pos"]], np.int32), g["base"], 1, 1, D, q_norm=w, k_norm=w, eps=c["eps"])
+
+
+def test_rope_hand_worked_fixture():
+    g = _load_rope_golden()
+    for c in g["cases"]:
+        Q, K, V = _rope_golden_case(oracle.qkv_rope, g, c)
+        assert np.allclose(Q[0, 0], c["q"], rtol=0, atol=g["tol"]), c["name"]
+        assert np.allclose(K[0, 0], c["q"], rtol=0, atol=g["tol"]), c["name"]
+        assert np.allclose(V[0, 0], c["v"], rtol=0, atol=g["tol"]), c["name"]
+
+
+def _proj_case(S, Hq, Hkv, D, d, seed):
+    x = _rand_bf16((S, d), seed)
+    Wq = _rand_bf16(((Hq + 2 * Hkv) * D, d), seed + 1, d ** -0.5)
+    qn = (1.0 + 0.25 * _rand_bf16((D,), seed + 2).float()).bfloat16()
+    kn = (1.0 + 0.25 * _rand_bf16((D,), seed + 3).float()).bfloat16()
+    return x, Wq, qn, kn
+
+
+@pytest.mark.parametrize("shift", [1000, 1 << 20])
+def test_rope_scores_depend_only_on_relative_position(shift):
+    """(R_p q) . (R_p' k) = q . R_(p'-p) k: shifting every position leaves every q.k unchanged."""
+    Hq, Hkv, D = 2, 1, 32
+    x, Wq, qn, kn = _proj_case(12, Hq, Hkv, D, 64, 31)
+    pos = np.sort(np.random.default_rng(0).choice(5000, 12, replace=False)).astype(np.int32)
+    Q0, K0, _ = oracle.qkv_rope(x, Wq, pos, 1e4, Hq, Hkv, D, qn, kn)
+    Q1, K1, _ = oracle.qkv_rope(x, Wq, pos + shift, 1e4, Hq, Hkv, D, qn, kn)
+    for h in range(Hq):
+        a, b = Q0[:, h] @ K0[:, 0].T, Q1[:, h] @ K1[:, 0].T
+        assert np.allclose(a, b, rtol=1e-9, atol=1e-9 * np.abs(a).max())
+    assert not np.allclose(Q0, Q1)  # the rotation itself did move
+
+
+def test_rope_preserves_head_norms_and_leaves_v_alone():
+    Hq, Hkv, D = 4, 2, 64
+    x, Wq, _, _ = _proj_case(10, Hq, Hkv, D, 64, 41)
+    pos = np.arange(10, dtype=np.int32) * 7919
+    Q0, K0, V0 = oracle.qkv_rope(x, Wq, np.zeros(10, np.int32), 1e6, Hq, Hkv, D)
+    Q1, K1, V1 = oracle.qkv_rope(x, Wq, pos, 1e6, Hq, Hkv, D)
+    assert np.allclose(np.linalg.norm(Q0, axis=-1), np.linalg.norm(Q1, axis=-1), rtol=1e-12)
+    assert np.allclose(np.linalg.norm(K0, axis=-1), np.linalg.norm(K1, axis=-1), rtol=1e-12)
+    half = D // 2  # each (j, j + D/2) pair keeps its own length
+    pair0 = Q0[..., :half] ** 2 + Q0[..., half:] ** 2
+    pair1 = Q1[..., :half] ** 2 + Q1[..., half:] ** 2
+    assert np.allclose(pair0, pair1, rtol=1e-10, atol=1e-12)
+    assert np.array_equal(V0, V1)
+
+
+def test_head_norm_is_per_head_and_scale_free():
+    Hq, Hkv, D = 4, 2, 32
+    x, Wq, _, _ = _proj_case(8, Hq, Hkv, D, 64, 51)
+    ones = _bf16(np.ones(D, np.float32))
+    pos = np.arange(8, dtype=np.int32) * 3
+    Q, K, _ = oracle.qkv_rope(x, Wq, pos, 1e6, Hq, Hkv, D, ones, ones, eps=0.0)
+    assert np.allclose(np.mean(Q ** 2, axis=-1), 1.0, rtol=1e-12)   # every head has unit RMS
+    assert np.allclose(np.mean(K ** 2, axis=-1), 1.0, rtol=1e-12)
+    Q4, K4, V4 = oracle.qkv_rope((x.float() * 4).bfloat16(), Wq, pos, 1e6, Hq, Hkv, D, ones, ones, eps=0.0)
+    assert np.allclose(Q4, Q, rtol=1e-12, atol=1e-12) and np.allclose(K4, K, rtol=1e-12, atol=1e-12)
+    _, _, V = oracle.qkv_rope(x, Wq, pos, 1e6, Hq, Hkv, D, ones, ones, eps=0.0)
+    assert np.allclose(V4, 4 * V, rtol=1e-12)
+
+
+def test_pruning_commutes_with_projection_at_original_positions():
+    """Projecting the kept rows at their original positions equals projecting the whole
+    prompt at positions 0..n-1 and keeping those rows."""
+    Hq, Hkv, D = 2, 1, 32
+    x, Wq, qn, kn = _proj_case(64, Hq, Hkv, D, 64, 61)
+    kept = np.sort(np.random.default_rng(1).choice(64, 20, replace=False)).astype(np.int32)
+    full = oracle.qkv_rope(x, Wq, np.arange(64, dtype=np.int32), 1e6, Hq, Hkv, D, qn, kn)
+    pruned = oracle.qkv_rope(x[torch.as_tensor(kept, dtype=torch.long)], Wq, kept, 1e6, Hq, Hkv, D, qn, kn)
+    for a, b in zip(full, pruned):
+        assert np.array_equal(a[kept], b)
+    rows = oracle.qkv_rope(x, Wq, np.arange(64, dtype=np.int32), 1e6, Hq, Hkv, D, qn, kn, rows=kept)
+    for a, b in zip(full, rows):
+        assert np.array_equal(a[kept], b)
