@@ -217,6 +217,49 @@ tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const t
                                     int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
                                     tg_bf16 *O, tg_stream stream);
 
+/* --------------------------------------------------------------------------
+ * tg_qkv_rope -- Q, K and V of a pruned layer, at the kept tokens' positions.
+ * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
+ * forward): the layers above the gate run on the kept tokens only, and each kept
+ * token stays at its prompt position.  On the article's Qwen3 backbone an
+ * attention block projects, normalises each Q / K head and applies the rotary
+ * embedding; for kept row i at position p = positions[i]:
+ *     y            = W_qkv hidden[i, :]                       (fp32 accumulation)
+ *     Q / K head u = y_head / sqrt(mean(y_head^2) + eps) * norm_weight
+ *                    (when q_norm / k_norm is NULL that head kind is not normalised)
+ *     phi_j        = p * rope_base^(-2j / D),   j < D/2
+ *     out_j        = u_j cos phi_j - u_(j+D/2) sin phi_j
+ *     out_(j+D/2)  = u_(j+D/2) cos phi_j + u_j sin phi_j
+ *     V head       = y_head (no norm, no rotation)
+ * One bf16 rounding at the end.
+ *
+ *   hidden    bf16 [S, d]                     W_qkv  bf16 [(Hq + 2 Hkv) D, d]
+ *             (rows: Hq Q heads, then Hkv K heads, then Hkv V heads)
+ *   positions int32 [S] (e.g. the kept indices from tg_select_topk)
+ *   q_norm, k_norm  bf16 [D] or NULL          eps    host float >= 0
+ *   Q bf16 [S, Hq, D]   Kc, V bf16 [S, Hkv, D]   (written, caller-allocated)
+ * Sizes: S >= 0; d a positive multiple of 8; D in {64, 128}; rope_base > 1.
+ * hidden, W_qkv, Q, Kc and V 16-byte aligned.
+ * -------------------------------------------------------------------------- */
+tg_status tg_qkv_rope(const tg_bf16 *hidden, int64_t S, int32_t d, const tg_bf16 *W_qkv,
+                      const int32_t *positions, double rope_base, const tg_bf16 *q_norm,
+                      const tg_bf16 *k_norm, float eps, int32_t Hq, int32_t Hkv, int32_t D,
+                      tg_bf16 *Q, tg_bf16 *Kc, tg_bf16 *V, tg_stream stream);
+
+/* --------------------------------------------------------------------------
+ * tg_linear -- the output projection of a pruned layer (o_proj), with the
+ * residual add fused: y[i, :] = W x[i, :] (+ residual[i, :]).
+ * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
+ * forward: the layers above the gate run on the kept tokens only).
+ *
+ *   x  bf16 [M, K]   W  bf16 [N, K] (nn.Linear layout)
+ *   residual bf16 [M, N] or NULL   y  bf16 [M, N] (written; may not alias x or W)
+ * Sizes: M >= 0; K a positive multiple of 8; N a positive multiple of 32.
+ * All pointers 16-byte aligned.  fp32 accumulation, one bf16 rounding.
+ * -------------------------------------------------------------------------- */
+tg_status tg_linear(const tg_bf16 *x, int64_t M, int32_t K, const tg_bf16 *W, int32_t N,
+                    const tg_bf16 *residual, tg_bf16 *y, tg_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

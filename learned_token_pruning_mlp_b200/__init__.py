@@ -4,7 +4,10 @@ The four calls (gate MLP scoring, top-K selection with the question kept, gather
 of the kept rows, token-gated causal GQA attention) run in hand-written CUDA
 kernels behind the C ABI of include/tokengate.h; this package is the thin
 ctypes binding over it (``_lib``) plus seeded synthetic workloads
-(``workloads``).  There is no CPU fallback.
+(``workloads``).  The projections around the attention of a pruned layer
+(QKV with per-head norm and rotary embedding at the kept tokens' positions, and
+the output projection with the residual add) sit behind the same ABI.  There is
+no CPU fallback.
 """
 from ._lib import (  # noqa: F401
     TG_DEVERR_BAD_SEQLENS,
@@ -20,7 +23,9 @@ from ._lib import (  # noqa: F401
     tg_gated_attention_varlen,
     tg_gather,
     tg_get_device_error,
+    tg_linear,
     tg_probe_wait_timeout,
+    tg_qkv_rope,
     tg_select_random_k,
     tg_select_topk,
     tg_select_topk_sweep,

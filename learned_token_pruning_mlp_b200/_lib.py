@@ -52,6 +52,9 @@ _SIGNATURES = {
     "tg_gated_attention": ([_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp, _vp], ctypes.c_int),
     "tg_gated_attention_varlen": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp, _vp],
                                   ctypes.c_int),
+    "tg_qkv_rope": ([_vp, _i64, _i32, _vp, _vp, ctypes.c_double, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
+                    ctypes.c_int),
+    "tg_linear": ([_vp, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
 }
 
 
@@ -225,3 +228,38 @@ def tg_gated_attention_varlen(Q, Kc, V, s, gain, tau: float, cu_seqlens, max_seq
         _dev(gain, torch.float32, "gain"), float(tau), _dev(cu_seqlens, torch.int32, "cu_seqlens"), B, total,
         int(max_seqlen), Hq, Hkv, D, _dev(O, bf, "O"), _stream(stream)))
     return O
+
+
+def tg_qkv_rope(hidden, W_qkv, positions, rope_base: float, Hq: int, Hkv: int, D: int, q_norm=None, k_norm=None,
+                eps: float = 1e-6, Q=None, Kc=None, V=None, stream=None):
+    S, d = hidden.shape
+    bf = torch.bfloat16
+    if Q is None:
+        Q = torch.empty((S, Hq, D), dtype=bf, device=hidden.device)
+    if Kc is None:
+        Kc = torch.empty((S, Hkv, D), dtype=bf, device=hidden.device)
+    if V is None:
+        V = torch.empty((S, Hkv, D), dtype=bf, device=hidden.device)
+    if W_qkv.shape != ((Hq + 2 * Hkv) * D, d):
+        raise ValueError(f"W_qkv must be [{(Hq + 2 * Hkv) * D}, {d}], got {tuple(W_qkv.shape)}")
+    if positions.numel() < S:
+        raise ValueError("positions needs one entry per row")
+    _check("tg_qkv_rope", lib().tg_qkv_rope(
+        _dev(hidden, bf, "hidden"), S, d, _dev(W_qkv, bf, "W_qkv"), _dev(positions, torch.int32, "positions"),
+        float(rope_base), _dev(q_norm, bf, "q_norm"), _dev(k_norm, bf, "k_norm"), float(eps), Hq, Hkv, D,
+        _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _stream(stream)))
+    return Q, Kc, V
+
+
+def tg_linear(x, W, residual=None, y=None, stream=None) -> torch.Tensor:
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    bf = torch.bfloat16
+    if y is None:
+        y = torch.empty((M, N), dtype=bf, device=x.device)
+    _check("tg_linear", lib().tg_linear(
+        _dev(x, bf, "x"), M, K, _dev(W, bf, "W"), N, _dev(residual, bf, "residual"), _dev(y, bf, "y"),
+        _stream(stream)))
+    return y

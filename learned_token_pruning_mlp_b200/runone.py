@@ -6,6 +6,8 @@
     python -m learned_token_pruning_mlp_b200.runone randomk --n 131072 --k 8192
     python -m learned_token_pruning_mlp_b200.runone sweep --n 131072 --k 8192   # budgets k/4, k/2, k, 2k
     python -m learned_token_pruning_mlp_b200.runone gather --n 131072 --rows 8704
+    python -m learned_token_pruning_mlp_b200.runone qkv --S 8704        # QKV + norm + rotary
+    python -m learned_token_pruning_mlp_b200.runone oproj --S 8704      # output projection + residual
 
 Each call is timed with CUDA events on the launching stream (after one warm-up
 call) and the mean per-call time is printed.  Shapes default to the 128k-context
@@ -25,7 +27,7 @@ from . import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention"])
+    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention", "qkv", "oproj"])
     ap.add_argument("--n", type=int, default=131072)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--h", type=int, default=256)
@@ -79,6 +81,21 @@ def main():
         hk = torch.empty(a.rows, a.d, dtype=torch.bfloat16, device=dev)
         sk = torch.empty(a.rows, dtype=torch.float32, device=dev)
         fn = lambda: tg.tg_gather(hidden, idx, hidden_k=hk, scores=sc, s_k=sk)
+    elif a.call == "qkv":
+        x = torch.randn(a.S, a.d, generator=g).to(torch.bfloat16).to(dev)
+        Wq = (torch.randn((a.hq + 2 * a.hkv) * a.D, a.d, generator=g) / math.sqrt(a.d)).to(torch.bfloat16).to(dev)
+        qn = torch.ones(a.D, dtype=torch.bfloat16, device=dev)
+        pos = torch.sort(torch.randperm(a.n, generator=g)[:a.S]).values.to(torch.int32).to(dev)
+        Q = torch.empty(a.S, a.hq, a.D, dtype=torch.bfloat16, device=dev)
+        K = torch.empty(a.S, a.hkv, a.D, dtype=torch.bfloat16, device=dev)
+        V = torch.empty_like(K)
+        fn = lambda: tg.tg_qkv_rope(x, Wq, pos, 1e6, a.hq, a.hkv, a.D, qn, qn, 1e-6, Q=Q, Kc=K, V=V)
+    elif a.call == "oproj":
+        x = torch.randn(a.S, a.hq * a.D, generator=g).to(torch.bfloat16).to(dev)
+        Wo = (torch.randn(a.d, a.hq * a.D, generator=g) / math.sqrt(a.hq * a.D)).to(torch.bfloat16).to(dev)
+        res = torch.randn(a.S, a.d, generator=g).to(torch.bfloat16).to(dev)
+        y = torch.empty(a.S, a.d, dtype=torch.bfloat16, device=dev)
+        fn = lambda: tg.tg_linear(x, Wo, res, y=y)
     else:
         Q = torch.randn(a.S, a.hq, a.D, generator=g).to(torch.bfloat16).to(dev)
         K = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
@@ -117,6 +134,10 @@ def main():
     if a.call == "attention":
         fl = 4 * a.D * a.hq * a.S * (a.S + 1) / 2
         extra = f" {fl / ms / 1e9:.1f} TFLOP/s"
+    elif a.call in ("qkv", "oproj"):
+        n_out = (a.hq + 2 * a.hkv) * a.D if a.call == "qkv" else a.d
+        k_in = a.d if a.call == "qkv" else a.hq * a.D
+        extra = f" {2 * a.S * n_out * k_in / ms / 1e9:.1f} TFLOP/s"
     print(f"{a.call}: {ms * 1e3:.1f} us per call{extra} (status bits {bits})")
     if bits:
         raise SystemExit(1)

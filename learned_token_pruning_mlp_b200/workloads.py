@@ -23,7 +23,7 @@ import torch
 _TAG = {
     "hidden": 1, "needles": 2, "w1": 3, "b1": 4, "w2": 5, "b2": 6,
     "gain": 7, "q": 8, "k": 9, "v": 10, "mix_base": 11, "mix_pick": 12,
-    "mix_tail": 13, "ties": 14, "sel": 15,
+    "mix_tail": 13, "ties": 14, "sel": 15, "wqkv": 16, "wo": 17, "qn": 18, "kn": 19,
 }
 
 
@@ -60,6 +60,8 @@ class Workload:
     needle_frac: float = 0.0          # share of document positions scaled x4
     score_mixture: bool = False       # selection scores drawn from N(0,1)+2% N(4,1)
     tau: float = 1.1
+    rope_base: float = 1e6            # Qwen3's rotary base
+    norm_eps: float = 1e-6            # Qwen3's RMS-norm epsilon
 
     @property
     def n(self) -> int:
@@ -195,3 +197,15 @@ def random_scores(n: int, seed: int) -> torch.Tensor:
     """fp32[n] ~ N(0,1): a generic key-bias vector for attention-only cases."""
     return torch.randn(n, generator=_gen(seed, "sel"), dtype=torch.float32)
 
+
+
+def layer_weights(w: Workload, layer: int = 0):
+    """Synthetic weights of one pruned attention layer, all bf16:
+    W_qkv [(hq + 2 hkv) D, d] ~ N(0, 1/d) (Q rows, then K rows, then V rows),
+    W_o [d, hq D] ~ N(0, 1/(hq D)), per-head norm weights q_norm, k_norm [D] ~ 1 + N(0, 0.1^2)."""
+    D = w.head_dim
+    W_qkv = _randn_bf16(((w.hq + 2 * w.hkv) * D, w.d), _gen(w.seed, "wqkv", layer), 1.0 / math.sqrt(w.d))
+    W_o = _randn_bf16((w.d, w.hq * D), _gen(w.seed, "wo", layer), 1.0 / math.sqrt(w.hq * D))
+    q_norm = (1.0 + 0.1 * torch.randn(D, generator=_gen(w.seed, "qn", layer))).to(torch.bfloat16)
+    k_norm = (1.0 + 0.1 * torch.randn(D, generator=_gen(w.seed, "kn", layer))).to(torch.bfloat16)
+    return W_qkv, W_o, q_norm, k_norm

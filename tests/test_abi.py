@@ -99,6 +99,25 @@ def test_attention_rejects_bad_arguments(L):
     assert L.tg_gated_attention_varlen(p, p, p, p, p, f, p, 2, 10, 11, 4, 2, 64, p, None) == 1
 
 
+def test_projections_reject_bad_arguments(L):
+    p = ctypes.c_void_p(4096)
+    f = ctypes.c_float(1e-6)
+    b = ctypes.c_double(1e6)
+    assert L.tg_linear(p, 10, 12, p, 64, None, p, None) == 2                               # K % 8
+    assert L.tg_linear(p, 10, 16, p, 48, None, p, None) == 2                               # N % 32
+    assert L.tg_linear(p, -1, 16, p, 64, None, p, None) == 1
+    assert L.tg_linear(p, 0, 16, p, 64, None, p, None) == 0                                # M = 0: no-op
+    assert L.tg_linear(None, 10, 16, p, 64, None, p, None) == 1
+    assert L.tg_linear(p, 10, 16, p, 64, ctypes.c_void_p(4098), p, None) == 3              # residual misaligned
+    assert L.tg_qkv_rope(p, 10, 64, p, p, b, None, None, f, 4, 2, 96, p, p, p, None) == 2  # D
+    assert L.tg_qkv_rope(p, 10, 60, p, p, b, None, None, f, 4, 2, 64, p, p, p, None) == 2  # d % 8
+    assert L.tg_qkv_rope(p, 10, 64, p, p, ctypes.c_double(1.0), None, None, f, 4, 2, 64, p, p, p, None) == 1
+    assert L.tg_qkv_rope(p, 10, 64, p, p, b, None, None, ctypes.c_float(-1.0), 4, 2, 64, p, p, p, None) == 1
+    assert L.tg_qkv_rope(p, 10, 64, p, None, b, None, None, f, 4, 2, 64, p, p, p, None) == 1
+    assert L.tg_qkv_rope(p, 0, 64, p, p, b, None, None, f, 4, 2, 64, p, p, p, None) == 0   # S = 0
+    assert L.tg_qkv_rope(p, 10, 64, p, p, b, None, None, f, 4, 2, 64, ctypes.c_void_p(4097), p, p, None) == 3
+
+
 def test_probe_rejects_bad_limit(L):
     assert L.tg_probe_wait_timeout(0, None) == 1
     assert L.tg_probe_wait_timeout(3_000_000_000, None) == 1
