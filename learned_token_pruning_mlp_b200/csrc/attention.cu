@@ -438,6 +438,13 @@ tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const fl
     const cudaError_t e = cudaFuncSetAttribute(gated_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    // the warpgroup register split in the kernel assumes 168 registers per thread at launch
+    cudaFuncAttributes fa;
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, gated_attention_kernel<D>);
+    if (ea != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(ea));
+    if (fa.numRegs != 168)
+      return tg::fail(TG_ERR_UNSUPPORTED, "gated_attention_kernel built with %d registers per thread; the register "
+                      "split needs 168", fa.numRegs);
     configured[dev] = true;
   }
   const float scale_log2 = tau / std::sqrt(static_cast<float>(D)) * kLog2e;

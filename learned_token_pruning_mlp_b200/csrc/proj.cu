@@ -12,14 +12,18 @@
 // B200 design: one CTA-pair tcgen05 GEMM (cta_group::2, 256 x 256 output tiles,
 // each CTA staging 128 rows of x and its half of the weight slice through 6 TMA
 // stages of 32 KB, double-buffered TMEM accumulators), persistent over tiles with
-// consecutive tiles sharing the same 256 rows of x.  The epilogue is where the
-// elementwise work goes: for the QKV projection a 256-column tile holds whole heads,
-// so each thread (one token row) has both halves (j, j + D/2) of every rotary pair in
-// its TMEM lane; it forms the angles pos * base^(-2j/D) in fp64 (exact reduction
-// modulo 2*pi even at positions of 2^31), takes sin/cos of the reduced angle, rotates,
-// rounds to bf16 and writes Q, K and V straight into their [S, H, D] buffers.  The
-// per-head norm needs the whole head row, which the same thread holds, so it costs
-// one pass over registers before the rotation.
+// consecutive tiles sharing the same 256 rows of x.  The elementwise work sits in the
+// epilogue, run by two warpgroups per CTA (each thread owns one row, i.e. one TMEM
+// lane, and half of the tile's columns):
+//   * output projection: + residual, whose rows are prefetched into L2 before the
+//     accumulator is ready;
+//   * QKV: a 256-column tile holds whole heads of one kind (Q, K or V).  The tile is
+//     four (head, 32-pair chunk) units; each warpgroup takes the two units that share
+//     one chunk of rotary indices j, so each thread forms 32 angles per tile and
+//     applies them to two heads.  The angle p * base^(-2j/D) is reduced modulo one
+//     turn exactly with a 64-bit fixed-point product (integer pipe), then sin/cos run
+//     in fp32.  The per-head norm takes the head's mean square in a first pass over
+//     TMEM.  Q, K and V go straight into their [S, H, D] buffers.
 #include <algorithm>
 #include <cmath>
 
@@ -32,7 +36,7 @@ constexpr int kBM = 128;         // rows per CTA (256 per pair)
 constexpr int kBN = 256;         // output columns per pair tile
 constexpr int kBK = 64;          // bf16 elements in one 128-byte swizzled row
 constexpr int kStages = 6;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warps 0-3: TMA, MMA, TMEM alloc, idle; 4-11: two epilogue warpgroups
 constexpr uint32_t kTileABytes = kBM * kBK * 2;          // 16 KB
 constexpr uint32_t kTileBBytes = (kBN / 2) * kBK * 2;    // 16 KB (this CTA's half)
 
@@ -64,7 +68,9 @@ struct ProjOut {
   const int32_t *pos;     // rotary position of every row
   int32_t q_cols;         // Hq * D
   int32_t k_cols;         // Hkv * D
-  double inv_freq[64];    // base^(-2j/D), j < D/2
+  // base^(-2j/D) / (2 pi) modulo 1 as a 64-bit binary fraction, j < D/2: the rotary
+  // angle of position p in turns is (p * turn[j] mod 2^64) / 2^64
+  uint64_t turn[64];
 };
 
 // Round 32 fp32 values to bf16 and write them as four 16-byte stores.
@@ -95,11 +101,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = tg::cluster_ctarank();
   const bool leader = rank == 0;
-  const int64_t pair = blockIdx.x >> 1;
-  const int64_t n_pairs = gridDim.x >> 1;
-  const int64_t m_tiles = (M + 2 * kBM - 1) / (2 * kBM);
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int n_pairs = static_cast<int>(gridDim.x >> 1);
+  const int m_tiles = static_cast<int>((M + 2 * kBM - 1) / (2 * kBM));
   const int n_tiles = (N + kBN - 1) / kBN;
-  const int64_t num_tiles = m_tiles * n_tiles;
+  const int num_tiles = m_tiles * n_tiles;  // below 2^31 (checked on the host)
   const int ksteps = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
@@ -109,7 +115,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tg::mbar_init(tg::smem_addr(&ctl->acc_full[a]), 1);
-      tg::mbar_init(tg::smem_addr(&ctl->acc_empty[a]), 2 * 128);
+      tg::mbar_init(tg::smem_addr(&ctl->acc_empty[a]), 2 * 256);
     }
     tg::mbar_init(tg::smem_addr(&ctl->drain), 1);
     ctl->abort_flag = 0;
@@ -128,22 +134,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tg::pdl_wait();
   tg::pdl_trigger();
   if (kHD > 0 && warp >= 4) {
-    for (int j = threadIdx.x - 128; j < kHD; j += 128) {
+    for (int j = threadIdx.x - 128; j < kHD; j += 256) {
       ctl->q_norm[j] = out.q_norm ? __bfloat162float(out.q_norm[j]) : 1.f;
       ctl->k_norm[j] = out.k_norm ? __bfloat162float(out.k_norm[j]) : 1.f;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+    asm volatile("bar.sync 1, 256;" ::: "memory");  // the two epilogue warpgroups
   }
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int *abort_flag = &ctl->abort_flag;
 
+  // Register split for the QKV epilogue (32 angles and two 32-wide TMEM rows live per
+  // thread): the launch gives 384 threads x 168 registers; 128 x 80 + 256 x 208 =
+  // 63488 <= 384 x 168, so the increase never waits (the launcher checks the launch
+  // count).
+  // Each warpgroup changes its budget inside its own branch.
+  if (warp < 4) {
+  if constexpr (kHD > 0) asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
     const uint64_t pol_a = tg::l2_policy_evict_last();  // x rows are reused by every N tile
     const uint64_t pol_b = tg::l2_policy_evict_last();  // the weights by every M tile
     uint32_t it = 0;
-    for (int64_t t = pair; t < num_tiles; t += n_pairs) {
-      const int64_t mt = t / n_tiles;
+    for (int t = pair; t < num_tiles; t += n_pairs) {
+      const int mt = t / n_tiles;
       const int nt = static_cast<int>(t % n_tiles);
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
         const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
@@ -163,7 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc = tg::idesc_bf16_f32(2 * kBM, kBN, false, false);
     uint32_t it = 0, tc = 0;
     bool ok = true;
-    for (int64_t t = pair; t < num_tiles && ok; t += n_pairs, ++tc) {
+    for (int t = pair; t < num_tiles && ok; t += n_pairs, ++tc) {
       const uint32_t acc = tc & 1u, aph = (tc >> 1) & 1u;
       if (!tg::mbar_wait(tg::smem_addr(&ctl->acc_empty[acc]), aph ^ 1u, abort_flag)) break;
       tg::tc_fence_after();
@@ -189,37 +202,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int local_abort = 0;
       tg::mbar_wait(tg::smem_addr(&ctl->drain), 0, &local_abort, 100000000ull);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    if constexpr (kHD > 0) asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
     // ---------------------------------------------------------------- epilogue (both CTAs)
-    const int quarter = warp - 4;
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. 32*quarter+31
+    const int group = (warp - 4) >> 2;     // 0 or 1: which half of the tile's work
     uint32_t tc = 0;
-    for (int64_t t = pair; t < num_tiles; t += n_pairs, ++tc) {
-      const int64_t mt = t / n_tiles;
+    for (int t = pair; t < num_tiles; t += n_pairs, ++tc) {
+      const int mt = t / n_tiles;
       const int nt = static_cast<int>(t % n_tiles);
       const uint32_t acc = tc & 1u, aph = (tc >> 1) & 1u;
-      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->acc_full[acc]), aph, abort_flag)) break;
-      tg::tc_fence_after();
-      const uint32_t taddr = tmem_base + acc * static_cast<uint32_t>(kBN) + (static_cast<uint32_t>(quarter * 32) << 16);
       const int64_t row = mt * 2 * kBM + rank * kBM + quarter * 32 + lane;
       const bool row_ok = row < M;
       const int n0 = nt * kBN;
       if constexpr (kHD == 0) {
+        // the residual slice this thread adds, pulled into L2 while the MMA runs
+        const int c0 = n0 + group * (kBN / 2);
+        if (out.residual && row_ok && c0 < N)
+          tg::prefetch_l2(out.residual + row * static_cast<int64_t>(N) + c0,
+                          static_cast<uint32_t>(min(kBN / 2, N - c0)) * 2u);
+      }
+      int32_t p = 0;
+      if constexpr (kHD > 0) p = row_ok ? out.pos[row] : 0;
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->acc_full[acc]), aph, abort_flag)) break;
+      tg::tc_fence_after();
+      const uint32_t taddr = tmem_base + acc * static_cast<uint32_t>(kBN) + (static_cast<uint32_t>(quarter * 32) << 16);
+      if constexpr (kHD == 0) {
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 0; c < kBN / 64; ++c) {
+          const int cc = group * (kBN / 64) + c;  // 32-column chunk of the tile
           uint32_t r[32];
-          tg::tmem_ld32(taddr + c * 32, r);
+          tg::tmem_ld32(taddr + cc * 32, r);
           tg::tmem_ld_wait();
-          const int col = n0 + c * 32;
+          const int col = n0 + cc * 32;
           if (row_ok && col < N) {
             float v[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (out.residual) {
               const uint4 *src = reinterpret_cast<const uint4 *>(out.residual + row * static_cast<int64_t>(N) + col);
+              uint4 u[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) u[q] = src[q];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const uint4 u = src[q];
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
@@ -234,11 +262,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       } else {
         constexpr int kHalf = kHD / 2;
-        const int32_t p = row_ok ? out.pos[row] : 0;
+        // units (head, chunk) of this warpgroup: two heads sharing rotary chunk jc
+        const int jc = kHD == 128 ? group : 0;                // chunk of 32 rotary indices
+        const int hA = kHD == 128 ? 0 : group;                // head offsets inside the tile
+        const int hB = kHD == 128 ? 1 : group + 2;
+        const int colA = n0 + hA * kHD, colB = n0 + hB * kHD;
+        // the 32 angles of this chunk, in turns, reduced exactly, then sin/cos
+        float cs[32], sn[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const uint64_t prod = static_cast<uint64_t>(static_cast<int64_t>(p)) * out.turn[32 * jc + e];
+          const uint32_t hi = static_cast<uint32_t>(prod >> 32);
+          float f = __uint_as_float(0x3F800000u | (hi >> 9)) - 1.0f;  // [0, 1) turns
+          f = f >= 0.5f ? f - 1.0f : f;                              // [-1/2, 1/2) turns
+          __sincosf(f * 6.28318530717958647692f, &sn[e], &cs[e]);
+        }
 #pragma unroll 1
-        for (int hd = 0; hd < kBN; hd += kHD) {
-          const int col = n0 + hd;  // first column of this head (warp-uniform)
+        for (int u = 0; u < 2; ++u) {
+          const int col = u == 0 ? colA : colB;  // warp-uniform
           if (col >= N) break;
+          const uint32_t hcol = static_cast<uint32_t>(col - n0);
           __nv_bfloat16 *dst;
           int64_t ld;
           const float *nw = nullptr;
@@ -255,60 +298,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             dst = out.v + (col - out.q_cols - out.k_cols);
             ld = out.k_cols;
           }
-          // pass 1 (normalised heads only): mean square of the head row
           float rn = 1.f;
-          if (nw) {
+          if (nw) {  // mean square of the whole head
             float ss = 0.f;
 #pragma unroll 1
             for (int c = 0; c < kHD / 32; ++c) {
               uint32_t r[32];
-              tg::tmem_ld32(taddr + hd + 32 * c, r);
+              tg::tmem_ld32(taddr + hcol + 32 * c, r);
               tg::tmem_ld_wait();
 #pragma unroll
               for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(r[e]), __uint_as_float(r[e]), ss);
             }
             rn = rsqrtf(ss * (1.0f / kHD) + out.eps);
           }
-          // pass 2: 32 rotary pairs (j, j + D/2) at a time
-          __nv_bfloat16 *drow = dst + row * ld;
-#pragma unroll 1
-          for (int c = 0; c < kHalf / 32; ++c) {
-            uint32_t lo[32], hi[32];
-            tg::tmem_ld32(taddr + hd + 32 * c, lo);
-            tg::tmem_ld32(taddr + hd + kHalf + 32 * c, hi);
-            tg::tmem_ld_wait();
-            float a[32], b[32];
+          uint32_t lo[32], hi[32];
+          tg::tmem_ld32(taddr + hcol + 32 * jc, lo);
+          tg::tmem_ld32(taddr + hcol + kHalf + 32 * jc, hi);
+          tg::tmem_ld_wait();
+          float a[32], b[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            a[e] = __uint_as_float(lo[e]);
+            b[e] = __uint_as_float(hi[e]);
+          }
+          if (nw) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              a[e] = __uint_as_float(lo[e]);
-              b[e] = __uint_as_float(hi[e]);
+              a[e] = a[e] * rn * nw[32 * jc + e];
+              b[e] = b[e] * rn * nw[kHalf + 32 * jc + e];
             }
-            if (nw) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                a[e] = a[e] * rn * nw[32 * c + e];
-                b[e] = b[e] * rn * nw[kHalf + 32 * c + e];
-              }
-            }
-            if (!is_v) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                // angle p * base^(-2j/D) reduced modulo 2*pi in fp64, then sin/cos in fp32
-                const double th = static_cast<double>(p) * out.inv_freq[32 * c + e];
-                const double red = th - 6.283185307179586476925 * rint(th * 0.159154943091895335769);
-                float sn, cs;
-                __sincosf(static_cast<float>(red), &sn, &cs);
-                const float x0 = a[e], x1 = b[e];
-                a[e] = x0 * cs - x1 * sn;
-                b[e] = x1 * cs + x0 * sn;
-              }
-            }
-            if (row_ok) {
-              store_row32(drow + 32 * c, a);
-              store_row32(drow + kHalf + 32 * c, b);
-            }
-            __syncwarp();
           }
+          if (!is_v) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x0 = a[e], x1 = b[e];
+              a[e] = x0 * cs[e] - x1 * sn[e];
+              b[e] = x1 * cs[e] + x0 * sn[e];
+            }
+          }
+          if (row_ok) {
+            __nv_bfloat16 *drow = dst + row * ld;
+            store_row32(drow + 32 * jc, a);
+            store_row32(drow + kHalf + 32 * jc, b);
+          }
+          __syncwarp();
         }
       }
       tg::tc_fence_before();
@@ -353,9 +386,19 @@ tg_status launch_proj(const tg_bf16 *x, int64_t M, int32_t K, const tg_bf16 *W, 
     const cudaError_t e =
         cudaFuncSetAttribute(proj_gemm_kernel<kHD>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (kHD > 0) {
+      // the register split in the kernel assumes 168 registers per thread at launch
+      cudaFuncAttributes fa;
+      const cudaError_t ea = cudaFuncGetAttributes(&fa, proj_gemm_kernel<kHD>);
+      if (ea != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(ea));
+      if (fa.numRegs != 168)
+        return tg::fail(TG_ERR_UNSUPPORTED, "%s built with %d registers per thread; the warpgroup register split "
+                        "needs 168", name, fa.numRegs);
+    }
     configured[dev] = true;
   }
   const int64_t tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kBN - 1) / kBN);
+  if (tiles > 0x7FFFFFFF) return tg::fail(TG_ERR_UNSUPPORTED, "%s: more than 2^31 - 1 output tiles", name);
   const int64_t pairs = std::min<int64_t>(tiles, tg::sm_count() / 2);
   const cudaError_t e = tg::launch_pdl(proj_gemm_kernel<kHD>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads),
                                       kSmem, stream, tm_a, tm_b, M, N, K, out, err);
@@ -410,7 +453,15 @@ extern "C" tg_status tg_qkv_rope(const tg_bf16 *hidden, int64_t S, int32_t d, co
   out.eps = eps;
   out.q_cols = Hq * D;
   out.k_cols = Hkv * D;
-  for (int j = 0; j < D / 2; ++j) out.inv_freq[j] = std::pow(rope_base, -2.0 * j / D);
+  // base^(-2j/D) / (2 pi) modulo 1 as a 64-bit binary fraction (x86 long double
+  // carries 64 significant bits, so the table is exact to about 2^-64 turns)
+  const long double two_pi = 6.283185307179586476925286766559005768L;
+  for (int j = 0; j < D / 2; ++j) {
+    long double g = std::pow(static_cast<long double>(rope_base), -2.0L * j / D) / two_pi;
+    g -= std::floor(g);
+    const long double scaled = std::ldexp(g, 64);
+    out.turn[j] = scaled >= 18446744073709551615.0L ? ~uint64_t(0) : static_cast<uint64_t>(scaled);
+  }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 64) return launch_proj<64>(hidden, S, d, W_qkv, static_cast<int32_t>(N), out, st, "proj_gemm_kernel<qkv64>");
   return launch_proj<128>(hidden, S, d, W_qkv, static_cast<int32_t>(N), out, st, "proj_gemm_kernel<qkv128>");
