@@ -45,6 +45,10 @@ def lib():
         L.orc_splitmix64.restype = ctypes.c_uint64
         L.orc_select_random_k.argtypes = [vp, i64, i64, ctypes.c_uint64, vp]
         L.orc_select_random_k.restype = i64
+        L.orc_gated_attention_lse_rows.argtypes = [vp, vp, vp, vp, f64, i32, i32, i32, vp, i64, vp]
+        L.orc_gated_attention_lse_rows.restype = None
+        L.orc_gated_attention_backward.argtypes = [vp, vp, vp, vp, vp, f64, vp, i64, i32, i32, i32, vp, vp, vp]
+        L.orc_gated_attention_backward.restype = None
         L.orc_qkv_rope_rows.argtypes = [vp, i32, vp, vp, f64, i32, i32, i32, vp, vp, f64, vp, i64, vp, vp, vp]
         L.orc_qkv_rope_rows.restype = None
         L.orc_linear_rows.argtypes = [vp, i32, vp, i32, vp, vp, i64, vp]
@@ -180,6 +184,35 @@ def gated_attention_varlen(Q, K, V, s, gain, tau: float, cu_seqlens: Sequence[in
         out[sel] = gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], _np(s, np.float32)[lo:hi], gain, tau,
                                    rows=rows_all[sel] - lo)
     return out
+
+
+def gated_attention_lse(Q, K, s, gain, tau: float, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """lse[r, h] = log sum_{j <= i} exp(tau*Q_ih.K_jg/sqrt(D) + gain_h*s_j), i = rows[r]; fp64 [R, Hq]."""
+    S, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    qb, kb = _bf16_bits(Q), _bf16_bits(K)
+    sv, gv = _np(s, np.float32), _np(gain, np.float32)
+    r = np.arange(S, dtype=np.int64) if rows is None else _np(rows, np.int64)
+    out = np.empty((len(r), Hq), dtype=np.float64)
+    lib().orc_gated_attention_lse_rows(_ptr(qb), _ptr(kb), _ptr(sv), _ptr(gv), float(tau), Hq, Hkv, D,
+                                       _ptr(r), len(r), _ptr(out))
+    return out
+
+
+def gated_attention_backward(Q, K, V, s, gain, tau: float, dO):
+    """Gradients of the loss with dL/dO = dO through token-gated attention:
+    (ds [S], dgain [Hq], dtau) in fp64, with dl_ij = P_ij (dO_i.V_j - dO_i.O_i),
+    ds_j = sum_{h,i} gain_h dl_ij, dgain_h = sum_{i,j} s_j dl_ij, dtau = sum dl_ij q_i.k_j/sqrt(D)."""
+    S, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    qb, kb, vb, db = _bf16_bits(Q), _bf16_bits(K), _bf16_bits(V), _bf16_bits(dO)
+    sv, gv = _np(s, np.float32), _np(gain, np.float32)
+    ds = np.empty(S, dtype=np.float64)
+    dg = np.empty(Hq, dtype=np.float64)
+    dt = np.empty(1, dtype=np.float64)
+    lib().orc_gated_attention_backward(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(sv), _ptr(gv), float(tau), _ptr(db),
+                                       S, Hq, Hkv, D, _ptr(ds), _ptr(dg), _ptr(dt))
+    return ds, dg, float(dt[0])
 
 
 # --------------------------------------------------------------------------- projections

@@ -26,6 +26,11 @@
  *                 additive key bias), row 0 = V[0], bias-shift invariance,
  *                 duplicated-KV-head equivalence, convex-hull bound,
  *                 pruned keys never influence an output.
+ *   backward   -- torch autograd in fp64 through an independent softmax
+ *                 attention, central finite differences of the forward above,
+ *                 a hand-worked two-token fixture, sum_j ds_j = 0 (a constant
+ *                 shift of every score leaves the softmax unchanged).
+ *   lse        -- torch logsumexp in fp64.
  *   projections -- torch fp64 matmul (positions 0, no norm), a hand-worked
  *                 rotary fixture, relative-position invariance of q.k, norm
  *                 preservation, scale invariance of the per-head norm, and
@@ -283,6 +288,132 @@ void orc_gated_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16
         free(q);
         free(l);
     }
+}
+
+/* ------------------------------------------------------------------------ *
+ * Log-sum-exp of each attention row (the normaliser of the softmax above):
+ *     lse[r, h] = log sum_{j <= i} exp(l_ij),   i = rows[r]
+ * with l_ij the token-gated logit defined above.  lse: double [n_rows, Hq].
+ * ------------------------------------------------------------------------ */
+void orc_gated_attention_lse_rows(const uint16_t *Q, const uint16_t *K, const float *s,
+                                  const float *gain, double tau, int32_t Hq, int32_t Hkv,
+                                  int32_t D, const int64_t *rows, int64_t n_rows, double *lse)
+{
+    const int32_t group = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < n_rows * Hq; ++t) {
+        const int64_t r = t / Hq;
+        const int32_t hh = (int32_t)(t % Hq);
+        const int64_t i = rows[r];
+        const int32_t g = hh / group;
+        const uint16_t *qi = Q + ((size_t)i * Hq + hh) * D;
+        double m = -INFINITY;
+        for (int pass = 0; pass < 2; ++pass) {
+            double sum = 0.0;
+            for (int64_t j = 0; j <= i; ++j) {
+                const uint16_t *kj = K + ((size_t)j * Hkv + g) * D;
+                double dot = 0.0;
+                for (int32_t c = 0; c < D; ++c) dot += bf16_value(qi[c]) * bf16_value(kj[c]);
+                const double l = tau * dot * inv_sqrt_d + (double)gain[hh] * (double)s[j];
+                if (pass == 0) {
+                    if (l > m) m = l;
+                } else {
+                    sum += exp(l - m);
+                }
+            }
+            if (pass == 1) lse[(size_t)r * Hq + hh] = m + log(sum);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ *
+ * Backward of token-gated attention with respect to the key scores, the per-head
+ * gains and the temperature: the gradient path from the attention layers back to
+ * the gate.  TokenGate article, "What is token-gated attention?": the gate score
+ * enters every layer above L as a logit bias with a learnable per-head gain and a
+ * learnable temperature, and the gate is trained through it.
+ * For an upstream gradient dO of the output O defined above (loss L with
+ * dL/dO = dO), per head h and query row i, with P_i. = softmax_j(l_i.), j <= i:
+ *     dP_ij    = dO[i,h,:] . V[j,g,:]
+ *     Delta_i  = sum_j P_ij dP_ij            (= dO_i . O_i)
+ *     dl_ij    = P_ij (dP_ij - Delta_i)     (dL/dl_ij through the softmax)
+ * and, since l_ij = tau (q_i . k_j)/sqrt(D) + gain_h s_j,
+ *     ds_j    += gain_h dl_ij
+ *     dgain_h += s_j dl_ij
+ *     dtau    += dl_ij (q_i . k_j) / sqrt(D)
+ * summed over every head h and row i.  dO: bf16 [S, Hq, D].  Outputs are double:
+ * ds [S], dgain [Hq], dtau [1].  Heads run in parallel into per-head buffers that
+ * are then added in head order.
+ * ------------------------------------------------------------------------ */
+void orc_gated_attention_backward(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                  const float *s, const float *gain, double tau,
+                                  const uint16_t *dO, int64_t S, int32_t Hq, int32_t Hkv,
+                                  int32_t D, double *ds, double *dgain, double *dtau)
+{
+    const int32_t group = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double *ds_h = (double *)calloc((size_t)Hq * (size_t)(S > 0 ? S : 1), sizeof(double));
+    double *dtau_h = (double *)calloc((size_t)Hq, sizeof(double));
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t hh = 0; hh < Hq; ++hh) {
+        const int32_t g = hh / group;
+        double *dsh = ds_h + (size_t)hh * (size_t)S;
+        double *l = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+        double *qk = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+        double dg = 0.0, dt = 0.0;
+        for (int64_t i = 0; i < S; ++i) {
+            const uint16_t *qi = Q + ((size_t)i * Hq + hh) * D;
+            const uint16_t *doi = dO + ((size_t)i * Hq + hh) * D;
+            double m = -INFINITY;
+            for (int64_t j = 0; j <= i; ++j) {
+                const uint16_t *kj = K + ((size_t)j * Hkv + g) * D;
+                const uint16_t *vj = V + ((size_t)j * Hkv + g) * D;
+                double dot = 0.0, dpv = 0.0;
+                for (int32_t c = 0; c < D; ++c) {
+                    dot += bf16_value(qi[c]) * bf16_value(kj[c]);
+                    dpv += bf16_value(doi[c]) * bf16_value(vj[c]);
+                }
+                qk[j] = dot * inv_sqrt_d;
+                dp[j] = dpv;
+                l[j] = tau * qk[j] + (double)gain[hh] * (double)s[j];
+                if (l[j] > m) m = l[j];
+            }
+            double denom = 0.0;
+            for (int64_t j = 0; j <= i; ++j) {
+                l[j] = exp(l[j] - m);  /* unnormalised weight */
+                denom += l[j];
+            }
+            double delta = 0.0;
+            for (int64_t j = 0; j <= i; ++j) {
+                l[j] /= denom;         /* P_ij */
+                delta += l[j] * dp[j];
+            }
+            for (int64_t j = 0; j <= i; ++j) {
+                const double dl = l[j] * (dp[j] - delta);
+                dsh[j] += (double)gain[hh] * dl;
+                dg += (double)s[j] * dl;
+                dt += dl * qk[j];
+            }
+        }
+        dgain[hh] = dg;
+        dtau_h[hh] = dt;
+        free(l);
+        free(qk);
+        free(dp);
+    }
+    double t = 0.0;
+    for (int32_t hh = 0; hh < Hq; ++hh) t += dtau_h[hh];
+    *dtau = t;
+    for (int64_t j = 0; j < S; ++j) {
+        double a = 0.0;
+        for (int32_t hh = 0; hh < Hq; ++hh) a += ds_h[(size_t)hh * (size_t)S + j];
+        ds[j] = a;
+    }
+    free(ds_h);
+    free(dtau_h);
 }
 
 /* ------------------------------------------------------------------------ *

@@ -170,3 +170,43 @@ def test_projection_pins_reject_planted_mistakes():
 
 def _bf16_ones(D):
     return torch.ones(D, dtype=torch.bfloat16)
+
+
+def _backward_variant(Q, K, V, dO, s, gain, tau, *, delta=True, gain_in_ds=True, sqrt_d=True, causal=True):
+    """A numpy copy of the score / gain / temperature backward with one planted mistake."""
+    q, kk, v, do = (t.double().numpy() for t in (Q, K, V, dO))
+    sv, gv = np.asarray(s, np.float64), np.asarray(gain, np.float64)
+    S, Hq, D = q.shape
+    Hkv = kk.shape[1]
+    ds, dg, dt = np.zeros(S), np.zeros(Hq), 0.0
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        qk = q[:, h] @ kk[:, g].T / math.sqrt(D)
+        L = tau * qk + gv[h] * sv[None, :]
+        if causal:
+            L = np.where(np.tril(np.ones((S, S), bool)), L, -np.inf)
+        P = np.exp(L - L.max(1, keepdims=True))
+        P /= P.sum(1, keepdims=True)
+        dP = do[:, h] @ v[:, g].T
+        dl = P * (dP - ((P * dP).sum(1, keepdims=True) if delta else 0.0))
+        ds += (gv[h] if gain_in_ds else 1.0) * dl.sum(0)
+        dg[h] = (dl * sv[None, :]).sum()
+        dt += (dl * (qk if sqrt_d else qk * math.sqrt(D))).sum()
+    return ds, dg, dt
+
+
+def test_backward_pins_reject_planted_mistakes():
+    from test_oracle_pins import _bwd_case, _autograd_backward
+    Q, K, V, dO, s, gain = _bwd_case(24, 4, 2, 16, 0)
+    tau = 1.1
+    ref = _autograd_backward(Q, K, V, dO, s, gain, tau)
+
+    def passes(**mut):
+        got = _backward_variant(Q, K, V, dO, s, gain, tau, **mut)
+        return all(np.allclose(a, b, rtol=1e-9, atol=1e-12) for a, b in zip(got, ref))
+
+    assert passes()                        # the unmutated copy passes
+    assert not passes(delta=False)         # softmax Jacobian without the Delta term
+    assert not passes(gain_in_ds=False)    # score gradient without the head's gain
+    assert not passes(sqrt_d=False)        # temperature gradient without 1/sqrt(D)
+    assert not passes(causal=False)        # keys after the query counted

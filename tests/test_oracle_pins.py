@@ -538,3 +538,113 @@ def test_pruning_commutes_with_projection_at_original_positions():
     rows = oracle.qkv_rope(x, Wq, np.arange(64, dtype=np.int32), 1e6, Hq, Hkv, D, qn, kn, rows=kept)
     for a, b in zip(full, rows):
         assert np.array_equal(a[kept], b)
+
+
+# ============================================================================ attention backward
+def _bwd_case(S, Hq, Hkv, D, seed, quant=False):
+    g = torch.Generator().manual_seed(seed)
+    Q = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    K = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    dO = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    s = torch.randn(S, generator=g)
+    gain = 0.5 + torch.rand(Hq, generator=g)
+    if quant:  # on a 2^-8 grid, so s +- 2^-10 and gain +- 2^-10 stay exact in fp32
+        s = torch.round(s * 256) / 256
+        gain = torch.round(gain * 256) / 256
+    return Q, K, V, dO, s, gain
+
+
+def _autograd_backward(Q, K, V, dO, s, gain, tau):
+    """Independent fp64 torch forward (explicit softmax over masked logits) and torch.autograd."""
+    q, k, v, do = (t.double() for t in (Q, K, V, dO))
+    S, Hq, D = q.shape
+    Hkv = k.shape[1]
+    sv = s.double().clone().requires_grad_(True)
+    gv = gain.double().clone().requires_grad_(True)
+    tv = torch.tensor(float(tau), dtype=torch.float64, requires_grad=True)
+    kk = k.repeat_interleave(Hq // Hkv, dim=1)
+    vv = v.repeat_interleave(Hq // Hkv, dim=1)
+    logits = tv * torch.einsum("ihd,jhd->hij", q, kk) / math.sqrt(D) + gv[:, None, None] * sv[None, None, :]
+    mask = torch.tril(torch.ones(S, S, dtype=torch.bool))
+    logits = logits.masked_fill(~mask, float("-inf"))
+    out = torch.einsum("hij,jhd->ihd", torch.softmax(logits, dim=-1), vv)
+    (out * do).sum().backward()
+    return sv.grad.numpy(), gv.grad.numpy(), float(tv.grad)
+
+
+@pytest.mark.parametrize("S,Hq,Hkv,D,tau,seed", [(24, 4, 2, 16, 1.1, 0), (40, 2, 1, 8, -0.7, 1), (17, 2, 2, 32, 0.0, 2)])
+def test_backward_matches_torch_autograd(S, Hq, Hkv, D, tau, seed):
+    Q, K, V, dO, s, gain = _bwd_case(S, Hq, Hkv, D, seed)
+    ds, dg, dt = oracle.gated_attention_backward(Q, K, V, s, gain, tau, dO)
+    rs, rg, rt = _autograd_backward(Q, K, V, dO, s, gain, tau)
+    assert np.allclose(ds, rs, rtol=1e-10, atol=1e-12)
+    assert np.allclose(dg, rg, rtol=1e-10, atol=1e-12)
+    assert math.isclose(dt, rt, rel_tol=1e-10, abs_tol=1e-12)
+
+
+def _loss(Q, K, V, dO, s, gain, tau):
+    """sum(dO * O) with O from the (separately pinned) forward oracle."""
+    return float(np.sum(dO.double().numpy() * oracle.gated_attention(Q, K, V, s, gain, tau)))
+
+
+def test_backward_matches_central_differences_of_the_forward():
+    Q, K, V, dO, s, gain = _bwd_case(16, 2, 1, 8, 5, quant=True)
+    tau = 0.9
+    ds, dg, dt = oracle.gated_attention_backward(Q, K, V, s, gain, tau, dO)
+    eps = 2.0 ** -10
+    for j in (0, 3, 9, 15):
+        e = torch.zeros_like(s)
+        e[j] = eps
+        fd = (_loss(Q, K, V, dO, s + e, gain, tau) - _loss(Q, K, V, dO, s - e, gain, tau)) / (2 * eps)
+        assert math.isclose(ds[j], fd, rel_tol=1e-4, abs_tol=1e-6), (j, ds[j], fd)
+    for h in range(2):
+        e = torch.zeros_like(gain)
+        e[h] = eps
+        fd = (_loss(Q, K, V, dO, s, gain + e, tau) - _loss(Q, K, V, dO, s, gain - e, tau)) / (2 * eps)
+        assert math.isclose(dg[h], fd, rel_tol=1e-4, abs_tol=1e-6), (h, dg[h], fd)
+    fd = (_loss(Q, K, V, dO, s, gain, tau + eps) - _loss(Q, K, V, dO, s, gain, tau - eps)) / (2 * eps)
+    assert math.isclose(dt, fd, rel_tol=1e-4, abs_tol=1e-6), (dt, fd)
+
+
+def test_backward_hand_worked_fixture():
+    with open(os.path.join(GOLDEN, "attention_backward_worked.json")) as f:
+        c = json.load(f)
+    S, Hq, Hkv, D = c["S"], c["Hq"], c["Hkv"], c["D"]
+    Q = _bf16(np.asarray(c["q"], np.float32).reshape(S, Hq, D))
+    K = _bf16(np.asarray(c["k"], np.float32).reshape(S, Hkv, D))
+    V = _bf16(np.asarray(c["v"], np.float32).reshape(S, Hkv, D))
+    dO = _bf16(np.asarray(c["dO"], np.float32).reshape(S, Hq, D))
+    ds, dg, dt = oracle.gated_attention_backward(Q, K, V, np.asarray(c["s"], np.float32),
+                                                 np.asarray(c["gain"], np.float32), c["tau"], dO)
+    assert np.allclose(ds, c["ds"], rtol=0, atol=c["tol"])
+    assert np.allclose(dg, c["dgain"], rtol=0, atol=c["tol"])
+    assert abs(dt - c["dtau"]) <= c["tol"]
+
+
+def test_backward_invariants():
+    Q, K, V, dO, s, gain = _bwd_case(30, 4, 2, 16, 7)
+    ds, dg, dt = oracle.gated_attention_backward(Q, K, V, s, gain, 1.3, dO)
+    # a constant added to every score leaves each softmax row unchanged
+    assert abs(ds.sum()) <= 1e-12 * np.abs(ds).sum()
+    # no gain: the scores do not reach the logits
+    ds0, _, _ = oracle.gated_attention_backward(Q, K, V, s, torch.zeros_like(gain), 1.3, dO)
+    assert np.all(ds0 == 0.0)
+    # no upstream gradient
+    z = oracle.gated_attention_backward(Q, K, V, s, gain, 1.3, torch.zeros_like(dO))
+    assert np.all(z[0] == 0) and np.all(z[1] == 0) and z[2] == 0
+    # the last token's score only reaches the last row
+    dsl, _, _ = oracle.gated_attention_backward(Q[-1:], K[-1:], V[-1:], s[-1:], gain, 1.3, dO[-1:])
+    assert dsl[0] == 0.0  # one key: softmax is constant
+
+
+def test_lse_matches_torch_logsumexp():
+    Q, K, _, _, s, gain = _bwd_case(33, 4, 2, 16, 9)
+    tau = 1.2
+    q, k = Q.double(), K.double().repeat_interleave(2, dim=1)
+    logits = tau * torch.einsum("ihd,jhd->hij", q, k) / 4.0 + gain.double()[:, None, None] * s.double()[None, None, :]
+    logits = logits.masked_fill(~torch.tril(torch.ones(33, 33, dtype=torch.bool)), float("-inf"))
+    ref = torch.logsumexp(logits, dim=-1).T.numpy()
+    assert np.allclose(oracle.gated_attention_lse(Q, K, s, gain, tau), ref, rtol=1e-12, atol=1e-12)
+    rows = [32, 0, 7]
+    assert np.allclose(oracle.gated_attention_lse(Q, K, s, gain, tau, rows=rows), ref[rows], rtol=1e-12, atol=1e-12)
