@@ -206,6 +206,17 @@ tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 
                              int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
                              tg_bf16 *O, tg_stream stream);
 
+/* The same forward for training: also stores what tg_gated_attention_backward
+ * needs.  lse[i * Hq + h] = log sum_{j <= i} exp(logit(i, j)) (natural log), fp32
+ * [S, Hq], required.  O32: fp32 [S, Hq, D] or NULL: the output before its bf16
+ * rounding; given to the backward, it keeps that rounding out of dO . O (at S =
+ * 8704 the rounding otherwise moves the first keys' score gradients by ~10 % of
+ * their rms).  Both caller-allocated, 16-byte aligned, written. */
+tg_status tg_gated_attention_train(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                   const float *s, const float *gain, float tau,
+                                   int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                   tg_bf16 *O, float *lse, float *O32, tg_stream stream);
+
 /* Packed ragged batch: request b owns rows [cu_seqlens[b], cu_seqlens[b+1]) of
  * Q, Kc, V, s and O (cu_seqlens: device int32 [B+1], e.g. cu_kept from
  * tg_select_topk_varlen) and attends causally within itself only.  total is
@@ -216,6 +227,41 @@ tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const t
                                     const int32_t *cu_seqlens, int32_t B, int64_t total,
                                     int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
                                     tg_bf16 *O, tg_stream stream);
+
+/* --------------------------------------------------------------------------
+ * tg_gated_attention_backward -- gradients of token-gated attention with respect
+ * to the key scores, the per-head gains and the temperature: the path by which
+ * the gate is trained through the layers above it.
+ * TokenGate article, "What is token-gated attention?": the score is a logit bias
+ * with a learnable per-head gain, the dot product a learnable temperature.  For a
+ * loss L with dL/dO = dO, per head h, query i and key j <= i (g = h / (Hq/Hkv)):
+ *     P_ij    = exp(logit(i, j) - lse[i, h])
+ *     dl_ij   = P_ij (dO[i,h,:] . V[j,g,:] - dO[i,h,:] . O[i,h,:])
+ *     ds[j]   = sum_{h,i} gain[h] dl_ij
+ *     dgain[h]= sum_{i,j} s[j] dl_ij
+ *     dtau    = sum_{h,i,j} dl_ij (Q[i,h,:] . Kc[j,g,:]) / sqrt(D)
+ *
+ *   Q, dO, O  bf16 [S, Hq, D]     Kc, V  bf16 [S, Hkv, D]     s fp32 [S]
+ *   gain fp32 [Hq]   tau (host)   lse fp32 [S, Hq], O, O32 (fp32 [S, Hq, D] or NULL):
+ *   from tg_gated_attention_train with the same inputs.  dO . O is taken from O32
+ *   when it is given (recommended), else from O (one of the two must be given).
+ *   ds fp32 [S], dgain fp32 [Hq], dtau fp32 [1]: written (overwritten, not added to).
+ *   workspace: device memory of at least tg_gated_attention_backward_workspace(S, Hq)
+ *   bytes, 16-byte aligned, owned by the caller, contents irrelevant on entry; the
+ *   call uses it until the stream reaches the end of the call.
+ * Sizes as for tg_gated_attention.  Results are deterministic (fixed summation
+ * order).  fp32 arithmetic over the bf16 inputs; the probabilities are recomputed
+ * in fp32 from lse.
+ * -------------------------------------------------------------------------- */
+size_t tg_gated_attention_backward_workspace(int64_t S, int32_t Hq);
+
+tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                      const float *s, const float *gain, float tau,
+                                      const tg_bf16 *O, const float *O32, const tg_bf16 *dO,
+                                      const float *lse,
+                                      int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                      float *ds, float *dgain, float *dtau,
+                                      void *workspace, size_t workspace_bytes, tg_stream stream);
 
 /* --------------------------------------------------------------------------
  * tg_qkv_rope -- Q, K and V of a pruned layer, at the kept tokens' positions.

@@ -20,6 +20,9 @@ from ._lib import (  # noqa: F401
     tg_abi_version,
     tg_gate_score,
     tg_gated_attention,
+    tg_gated_attention_backward,
+    tg_gated_attention_backward_workspace,
+    tg_gated_attention_train,
     tg_gated_attention_varlen,
     tg_gather,
     tg_get_device_error,

@@ -52,6 +52,11 @@ _SIGNATURES = {
     "tg_gated_attention": ([_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp, _vp], ctypes.c_int),
     "tg_gated_attention_varlen": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp, _vp],
                                   ctypes.c_int),
+    "tg_gated_attention_train": ([_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
+                                 ctypes.c_int),
+    "tg_gated_attention_backward_workspace": ([_i64, _i32], ctypes.c_size_t),
+    "tg_gated_attention_backward": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp,
+                                     _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "tg_qkv_rope": ([_vp, _i64, _i32, _vp, _vp, ctypes.c_double, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
                     ctypes.c_int),
     "tg_linear": ([_vp, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
@@ -213,6 +218,53 @@ def tg_gated_attention(Q, Kc, V, s, gain, tau: float, O=None, stream=None) -> to
         _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _dev(s, torch.float32, "s"),
         _dev(gain, torch.float32, "gain"), float(tau), S, Hq, Hkv, D, _dev(O, bf, "O"), _stream(stream)))
     return O
+
+
+def tg_gated_attention_train(Q, Kc, V, s, gain, tau: float, O=None, lse=None, O32=None, keep_fp32=True,
+                             stream=None):
+    """Forward for training: returns (O bf16, lse fp32 [S, Hq], O32 fp32 [S, Hq, D] or None)."""
+    S, Hq, D = Q.shape
+    Hkv = Kc.shape[1]
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=Q.device)
+    if O32 is None and keep_fp32:
+        O32 = torch.empty((S, Hq, D), dtype=torch.float32, device=Q.device)
+    bf = torch.bfloat16
+    _check("tg_gated_attention_train", lib().tg_gated_attention_train(
+        _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _dev(s, torch.float32, "s"),
+        _dev(gain, torch.float32, "gain"), float(tau), S, Hq, Hkv, D, _dev(O, bf, "O"),
+        _dev(lse, torch.float32, "lse"), _dev(O32, torch.float32, "O32"), _stream(stream)))
+    return O, lse, O32
+
+
+def tg_gated_attention_backward_workspace(S: int, Hq: int) -> int:
+    return int(lib().tg_gated_attention_backward_workspace(int(S), int(Hq)))
+
+
+def tg_gated_attention_backward(Q, Kc, V, s, gain, tau: float, O, dO, lse, O32=None, ds=None, dgain=None,
+                                dtau=None, workspace=None, stream=None):
+    S, Hq, D = Q.shape
+    Hkv = Kc.shape[1]
+    dev = gain.device
+    if ds is None:
+        ds = torch.empty(S, dtype=torch.float32, device=dev)
+    if dgain is None:
+        dgain = torch.empty(Hq, dtype=torch.float32, device=dev)
+    if dtau is None:
+        dtau = torch.empty(1, dtype=torch.float32, device=dev)
+    need = tg_gated_attention_backward_workspace(S, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    bf = torch.bfloat16
+    _check("tg_gated_attention_backward", lib().tg_gated_attention_backward(
+        _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _dev(s, torch.float32, "s"),
+        _dev(gain, torch.float32, "gain"), float(tau), _dev(O, bf, "O"), _dev(O32, torch.float32, "O32"),
+        _dev(dO, bf, "dO"), _dev(lse, torch.float32, "lse"), S, Hq, Hkv, D, _dev(ds, torch.float32, "ds"),
+        _dev(dgain, torch.float32, "dgain"), _dev(dtau, torch.float32, "dtau"),
+        _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)))
+    return ds, dgain, dtau
 
 
 def tg_gated_attention_varlen(Q, Kc, V, s, gain, tau: float, cu_seqlens, max_seqlen: int, O=None,

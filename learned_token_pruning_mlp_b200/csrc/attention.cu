@@ -38,7 +38,10 @@
 //     rescaled in TMEM after P is stored (S_t(j) completing orders this after O_t's
 //     previous product).  Otherwise exponentials are taken against the stale max,
 //     which stays exact in fp32 and loses nothing in bf16.
-//   * The epilogue divides O by the row sum, converts to bf16 and stores the rows.
+//   * The epilogue divides O by the row sum, converts to bf16 and stores the rows;
+//     for training it also stores each row's log-sum-exp (natural log), from which
+//     the backward recomputes the probabilities, and optionally the output before its
+//     bf16 rounding (fp32), from which the backward forms dO . O.
 //   * CTAs are ordered heaviest first (the longest causal rows), which the hardware
 //     block scheduler turns into a longest-processing-time schedule.
 #include <algorithm>
@@ -93,7 +96,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ key_scores,
                            const float *__restrict__ gain, float scale_log2, const int32_t *__restrict__ cu_seqlens,
                            int64_t S_single, int64_t total, int n_mblocks, int B, int Hq, int Hkv,
-                           __nv_bfloat16 *__restrict__ O, uint32_t *err) {
+                           __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, float *__restrict__ O32,
+                           uint32_t *err) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -381,6 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::tc_fence_after();
       const float inv_l = 1.0f / l;
       const int64_t row = rt + r;
+      // base-2 log of sum_j 2^(eff S'_j) is eff m + log2 l (m the max the weights used)
+      if (lse && row < len) lse[(seg_start + row) * Hq + h] = (m * eff + __log2f(l)) * 0.6931471805599453f;
       __nv_bfloat16 *orow = O + ((seg_start + row) * Hq + h) * static_cast<int64_t>(D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -391,6 +397,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (O32 && row < len) {
+          float4 *d32 = reinterpret_cast<float4 *>(O32 + ((seg_start + row) * Hq + h) * static_cast<int64_t>(D) + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            d32[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                                 __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+        }
         if (row < len) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
@@ -412,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain, float tau,
                  const int32_t *cu_seqlens, int32_t B, int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv,
-                 tg_bf16 *O, cudaStream_t stream, uint32_t *err) {
+                 tg_bf16 *O, float *lse, float *O32, cudaStream_t stream, uint32_t *err) {
   using C = Cfg<D>;
   CUtensorMap tm_q, tm_k, tm_v;
   {
@@ -455,7 +468,7 @@ tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const fl
   const cudaError_t e = tg::launch_pdl(gated_attention_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
                                       C::kSmem, stream, tm_q, tm_k, tm_v, s, gain, scale_log2, cu_seqlens,
                                       cu_seqlens ? int64_t(0) : total, total, n_mblocks, B, Hq, Hkv,
-                                      reinterpret_cast<__nv_bfloat16 *>(O), err);
+                                      reinterpret_cast<__nv_bfloat16 *>(O), lse, O32, err);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gated_attention_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("gated_attention_kernel");
 }
@@ -486,8 +499,23 @@ extern "C" tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, con
   uint32_t *err = tg::device_error_word();
   if (!err) return TG_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, cs, err)
-                  : launch<64>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, cs, err);
+  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, nullptr, nullptr, cs, err)
+                  : launch<64>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, nullptr, nullptr, cs, err);
+}
+
+extern "C" tg_status tg_gated_attention_train(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
+                                              const float *gain, float tau, int64_t S, int32_t Hq, int32_t Hkv,
+                                              int32_t D, tg_bf16 *O, float *lse, float *O32, tg_stream stream) {
+  tg::clear_detail();
+  tg_status st = validate(Q, Kc, V, s, gain, tau, S, Hq, Hkv, D, O);
+  if (st != TG_OK || S == 0) return st;
+  if (!lse) return tg::fail(TG_ERR_INVALID_ARG, "lse is NULL");
+  if (O32 && !tg::aligned16(O32)) return tg::fail(TG_ERR_ALIGNMENT, "O32 must be 16-byte aligned");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, lse, O32, cs, err)
+                  : launch<64>(Q, Kc, V, s, gain, tau, nullptr, 1, S, S, Hq, Hkv, O, lse, O32, cs, err);
 }
 
 extern "C" tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
@@ -503,6 +531,6 @@ extern "C" tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *
   uint32_t *err = tg::device_error_word();
   if (!err) return TG_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, cs, err)
-                  : launch<64>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, cs, err);
+  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, nullptr, nullptr, cs, err)
+                  : launch<64>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, nullptr, nullptr, cs, err);
 }

@@ -1,0 +1,491 @@
+// attention_bwd.cu -- tg_gated_attention_backward: gradients of token-gated attention
+// with respect to the key scores s, the per-head gains and the temperature (the path
+// by which the gate learns through the layers above it).
+//
+// TokenGate article, "What is token-gated attention?": the gate score of every kept
+// token is a bias on the attention logits, scaled by a learnable per-head gain, and
+// the dot product carries a learnable temperature.  For a loss L with dL/dO = dO,
+// per head h (KV head g = h / (Hq/Hkv)), query i and key j <= i:
+//     P_ij    = exp(l_ij - lse_i)           lse_i from the forward
+//     dP_ij   = dO_i . V_j,   Delta_i = dO_i . O_i,   dl_ij = P_ij (dP_ij - Delta_i)
+//     ds_j    = sum_{h,i} gain_h dl_ij
+//     dgain_h = sum_{i,j} s_j dl_ij
+//     dtau    = sum_{h,i,j} dl_ij (q_i . k_j) / sqrt(D)
+//
+// B200 design, three kernels on the caller's stream (programmatic launches):
+//   1. prep: Delta_i = dO_i . O_i (from the forward's fp32 output when the caller has
+//      it, else from the bf16 output) and the base-2 lse of every (row, head), negated,
+//      into per-head vectors of the workspace padded to a multiple of 128 rows
+//      (padding: -lse = -inf and -Delta = 0, so padding queries contribute nothing).
+//   2. main, one CTA per (128-key block, head), heaviest (first) key blocks first.
+//      Keys sit on the TMEM lanes, so each thread owns one key and every sum over
+//      queries is a register sum.  Per 128-query block, from the diagonal on:
+//          S^T  = K Q^T    and    dP^T = V dO^T
+//      (tcgen05, M = 128 keys, N = 128 queries, K = D, operands K-major in shared
+//      memory) go to one of two TMEM buffers while two warpgroups (64 query columns
+//      each) form p = exp2(S c + b_j - lse2_i) with c = tau log2(e) / sqrt(D) and
+//      b_j = gain_h log2(e) s_j, dl = p (dP - Delta_i), and accumulate sum_i dl and
+//      sum_i dl S with packed f32x2 arithmetic.  Q and dO stream through a TMA
+//      pipeline, the lse / Delta vectors through bulk copies.
+//   3. reduce: ds, dgain and dtau from the per-(head, key) column sums and the
+//      per-CTA temperature partials, each summed in a fixed order, so the result is
+//      deterministic.
+#include <algorithm>
+#include <cmath>
+
+#include "ptx.cuh"
+#include "runtime.h"
+
+namespace {
+
+constexpr int kBK = 128;          // keys per CTA (TMEM lanes)
+constexpr int kBQ = 128;          // queries per step (TMEM columns of S^T and dP^T)
+constexpr int kThreads = 384;     // warps 0-3: TMA, MMA, TMEM alloc, idle; 4-11: two warpgroups
+constexpr int kAux = 4;           // stages of the lse / Delta vectors
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kHalfBytes = 128 * 64 * 2;  // 128 rows x 64 bf16 columns, 128-byte swizzle
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr uint32_t kTileBytes = kHalfBytes * kHalves;  // 128 rows x D bf16
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr size_t kSmem = 1024 + 2 * static_cast<size_t>(kTileBytes) +
+                                  2 * static_cast<size_t>(kStages) * kTileBytes + kAux * 2 * kBQ * 4 + kBK * 4 + 512;
+};
+
+struct BwdCtl {
+  uint64_t kv_full;
+  uint64_t q_full[4];
+  uint64_t q_empty[4];
+  uint64_t aux_full[kAux];
+  uint64_t aux_empty[kAux];
+  uint64_t s_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float tau_part[8];
+};
+
+// Workspace (fp32): -lse2 [Hq][S_pad], -Delta [Hq][S_pad], colsum [Hq][S_pad], tau partials [Hq][n_kb].
+struct Workspace {
+  float *nlse2, *ndelta, *colsum, *taup;
+};
+
+__host__ __device__ inline int64_t padded_rows(int64_t S) { return (S + kBK - 1) / kBK * kBK; }
+
+inline size_t workspace_bytes(int64_t S, int32_t Hq) {
+  const int64_t sp = padded_rows(S);
+  const size_t floats = static_cast<size_t>(Hq) * (3 * static_cast<size_t>(sp) + static_cast<size_t>(sp / kBK));
+  return (floats * 4 + 255) / 256 * 256;
+}
+
+inline Workspace carve(void *base, int64_t S, int32_t Hq) {
+  const size_t sp = static_cast<size_t>(padded_rows(S));
+  float *f = static_cast<float *>(base);
+  return Workspace{f, f + Hq * sp, f + 2 * Hq * sp, f + 3 * Hq * sp};
+}
+
+// ------------------------------------------------------------------------------ prep
+// One warp per (row, head) of the padded range: Delta = dO . O (fp32), and
+// the lse converted to base 2; both stored negated, per head.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16 *__restrict__ O,
+                                                            const float *__restrict__ O32,
+                                                            const __nv_bfloat16 *__restrict__ dO,
+                                                            const float *__restrict__ lse, int64_t S, int64_t S_pad,
+                                                            int Hq, Workspace ws) {
+  tg::pdl_wait();
+  tg::pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t n_rows = S_pad * Hq;
+  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < n_rows;
+       w += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t i = w / Hq;
+    const int h = static_cast<int>(w % Hq);
+    float nd = 0.f, nl = -INFINITY;
+    if (i < S) {
+      constexpr int kPer = D / 32;  // bf16 elements per lane (2 or 4)
+      const __nv_bfloat16 *d = dO + (i * Hq + h) * D + lane * kPer;
+      float acc = 0.f;
+      if (O32) {
+        const float *o32 = O32 + (i * Hq + h) * D + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; e += 2) {
+          const float2 a = *reinterpret_cast<const float2 *>(o32 + e);
+          const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(d + e);
+          acc = fmaf(a.x, __low2float(b), acc);
+          acc = fmaf(a.y, __high2float(b), acc);
+        }
+      } else {
+        const __nv_bfloat16 *o = O + (i * Hq + h) * D + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; e += 2) {
+          const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(o + e);
+          const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(d + e);
+          acc = fmaf(__low2float(a), __low2float(b), acc);
+          acc = fmaf(__high2float(a), __high2float(b), acc);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+      nd = -acc;
+      nl = -lse[i * Hq + h] * kLog2e;
+    }
+    if (lane == 0) {
+      ws.ndelta[h * S_pad + i] = nd;
+      ws.nlse2[h * S_pad + i] = nl;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ main
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const float *__restrict__ key_scores, const float *__restrict__ gain, float c_log2, int64_t S,
+                    int64_t S_pad, int Hq, int Hkv, Workspace ws, uint32_t *err) {
+  using C = BwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sK = smem;
+  uint8_t *sV = sK + C::kTileBytes;
+  uint8_t *sQ = sV + C::kTileBytes;                  // [NS][tile]
+  uint8_t *sdO = sQ + NS * C::kTileBytes;            // [NS][tile]
+  float *sL = reinterpret_cast<float *>(sdO + NS * C::kTileBytes);  // [kAux][kBQ]  -lse2
+  float *sDl = sL + kAux * kBQ;                                      // [kAux][kBQ]  -Delta
+  float *sCs = sDl + kAux * kBQ;                                     // [kBK] second warpgroup's column sums
+  BwdCtl *ctl = reinterpret_cast<BwdCtl *>(sCs + kBK);
+
+  const int n_kb = static_cast<int>(S_pad / kBK);
+  const int kb = static_cast<int>(blockIdx.x) / Hq;  // ascending: the longest key blocks first
+  const int h = static_cast<int>(blockIdx.x) % Hq;
+  const int g = h / (Hq / Hkv);
+  const int n_steps = n_kb - kb;                     // query blocks kb .. n_kb-1
+  const int warp = tg::warp_id();
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tg::mbar_init(tg::smem_addr(&ctl->kv_full), 1);
+    for (int s = 0; s < NS; ++s) {
+      tg::mbar_init(tg::smem_addr(&ctl->q_full[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->q_empty[s]), 1);
+    }
+    for (int a = 0; a < kAux; ++a) {
+      tg::mbar_init(tg::smem_addr(&ctl->aux_full[a]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->aux_empty[a]), 8);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tg::mbar_init(tg::smem_addr(&ctl->s_full[b]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->tmem_empty[b]), 256);
+    }
+    tg::mbar_init(tg::smem_addr(&ctl->drain), 1);
+    ctl->abort_flag = 0;
+    tg::fence_mbar_init();
+    tg::prefetch_tmap(&tm_q);
+    tg::prefetch_tmap(&tm_k);
+    tg::prefetch_tmap(&tm_v);
+    tg::prefetch_tmap(&tm_do);
+  }
+  if (warp == 2) {
+    tg::tmem_alloc(tg::smem_addr(&ctl->tmem_base), 512);
+    tg::tmem_relinquish();
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  tg::tc_fence_after();
+  tg::pdl_wait();
+  tg::pdl_trigger();
+  const uint32_t tmem_base = ctl->tmem_base;
+  volatile int *abort_flag = &ctl->abort_flag;
+
+  // Register split: the launch gives 384 threads x 168 registers; 128 x 80 + 256 x 208 =
+  // 63488 <= 384 x 168, so the increase never waits (the launcher checks the launch
+  // count).  Each warpgroup changes its budget inside its own branch.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA / bulk producer
+    const uint32_t kvb = tg::smem_addr(&ctl->kv_full);
+    tg::mbar_arrive_expect_tx(kvb, 2 * C::kTileBytes);
+    for (int hf = 0; hf < C::kHalves; ++hf) {
+      tg::tma_load_3d(tg::smem_addr(sK + hf * kHalfBytes), &tm_k, kvb, hf * 64, g, kb * kBK);
+      tg::tma_load_3d(tg::smem_addr(sV + hf * kHalfBytes), &tm_v, kvb, hf * 64, g, kb * kBK);
+    }
+    for (int n = 0; n < n_steps; ++n) {
+      const int qrow = (kb + n) * kBQ;
+      const int s = n % NS;
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->q_empty[s]), ((n / NS) & 1) ^ 1, abort_flag)) break;
+      const uint32_t qf = tg::smem_addr(&ctl->q_full[s]);
+      tg::mbar_arrive_expect_tx(qf, 2 * C::kTileBytes);
+      for (int hf = 0; hf < C::kHalves; ++hf) {
+        tg::tma_load_3d(tg::smem_addr(sQ + s * C::kTileBytes + hf * kHalfBytes), &tm_q, qf, hf * 64, h, qrow);
+        tg::tma_load_3d(tg::smem_addr(sdO + s * C::kTileBytes + hf * kHalfBytes), &tm_do, qf, hf * 64, h, qrow);
+      }
+      const int a = n % kAux;
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->aux_empty[a]), ((n / kAux) & 1) ^ 1, abort_flag)) break;
+      const uint32_t af = tg::smem_addr(&ctl->aux_full[a]);
+      tg::mbar_arrive_expect_tx(af, 2 * kBQ * 4);
+      tg::bulk_load(tg::smem_addr(sL + a * kBQ), ws.nlse2 + h * S_pad + qrow, kBQ * 4, af);
+      tg::bulk_load(tg::smem_addr(sDl + a * kBQ), ws.ndelta + h * S_pad + qrow, kBQ * 4, af);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = tg::idesc_bf16_f32(kBK, kBQ, false, false);
+    bool ok = tg::mbar_wait(tg::smem_addr(&ctl->kv_full), 0, abort_flag);
+    for (int n = 0; n < n_steps && ok; ++n) {
+      const int s = n % NS;
+      const int buf = n & 1;
+      if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->q_full[s]), (n / NS) & 1, abort_flag))) break;
+      if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->tmem_empty[buf]), ((n >> 1) & 1) ^ 1, abort_flag))) break;
+      tg::tc_fence_after();
+      const uint32_t d_s = tmem_base + static_cast<uint32_t>(buf * 256);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
+        tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(tg::smem_addr(sK) + off, 16, 1024),
+                        tg::smem_desc_sw128(tg::smem_addr(sQ + s * C::kTileBytes) + off, 16, 1024), idesc,
+                        kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
+        tg::mma_bf16_ss(d_s + kBQ, tg::smem_desc_sw128(tg::smem_addr(sV) + off, 16, 1024),
+                        tg::smem_desc_sw128(tg::smem_addr(sdO + s * C::kTileBytes) + off, 16, 1024), idesc,
+                        kk > 0 ? 1u : 0u);
+      }
+      tg::mma_commit(tg::smem_addr(&ctl->s_full[buf]));
+      tg::mma_commit(tg::smem_addr(&ctl->q_empty[s]));
+    }
+    if (*abort_flag) {
+      tg::mma_commit(tg::smem_addr(&ctl->drain));
+      int local_abort = 0;
+      tg::mbar_wait(tg::smem_addr(&ctl->drain), 0, &local_abort, 100000000ull);
+    }
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    // ------------------------------------------------------------ dl and its sums
+    const int grp = (warp - 4) >> 2;       // query columns 64*grp .. 64*grp+63
+    const int quarter = warp & 3;          // TMEM lane quarter
+    const int r = quarter * 32 + lane;     // key within the block
+    const int64_t j = static_cast<int64_t>(kb) * kBK + r;
+    const float bj = j < S ? gain[h] * kLog2e * key_scores[j] : -INFINITY;
+    const uint64_t bj2 = tg::f2_pack(bj, bj);
+    const uint64_t c2 = tg::f2_pack(c_log2, c_log2);
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint64_t cs2 = tg::f2_pack(0.f, 0.f), ta2 = tg::f2_pack(0.f, 0.f);
+    for (int n = 0; n < n_steps; ++n) {
+      const int buf = n & 1;
+      const int a = n % kAux;
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->s_full[buf]), (n >> 1) & 1, abort_flag)) break;
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->aux_full[a]), (n / kAux) & 1, abort_flag)) break;
+      tg::tc_fence_after();
+      const uint32_t t_s = tmem_base + static_cast<uint32_t>(buf * 256 + 64 * grp) + lane_off;
+      uint32_t sx[64], dp[64];
+      tg::tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sx[0]));
+      tg::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sx[32]));
+      tg::tmem_ld32(t_s + kBQ, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tg::tmem_ld32(t_s + kBQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tg::tmem_ld_wait();
+      tg::tc_fence_before();
+      tg::mbar_arrive(tg::smem_addr(&ctl->tmem_empty[buf]));
+      const uint64_t *nl = reinterpret_cast<const uint64_t *>(sL + a * kBQ + 64 * grp);
+      const uint64_t *nd = reinterpret_cast<const uint64_t *>(sDl + a * kBQ + 64 * grp);
+      const bool diag = n == 0;  // query block == key block: keep query >= key
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const uint64_t s2 = tg::f2_pack(__uint_as_float(sx[2 * c]), __uint_as_float(sx[2 * c + 1]));
+        const uint64_t x2 = tg::f2_fma(s2, c2, tg::f2_add(bj2, nl[c]));
+        float x0, x1;
+        tg::f2_unpack(x2, x0, x1);
+        if (diag) {
+          const int q0 = 64 * grp + 2 * c;
+          if (q0 < r) x0 = -INFINITY;
+          if (q0 + 1 < r) x1 = -INFINITY;
+        }
+        const uint64_t p2 = tg::f2_pack(tg::ex2_approx(x0), tg::ex2_approx(x1));
+        const uint64_t d2 = tg::f2_add(tg::f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])), nd[c]);
+        const uint64_t dl2 = tg::f2_mul(p2, d2);
+        cs2 = tg::f2_add(cs2, dl2);
+        ta2 = tg::f2_fma(dl2, s2, ta2);
+      }
+      __syncwarp();
+      if (lane == 0) tg::mbar_arrive(tg::smem_addr(&ctl->aux_empty[a]));
+    }
+    float cs0, cs1, ta0, ta1;
+    tg::f2_unpack(cs2, cs0, cs1);
+    tg::f2_unpack(ta2, ta0, ta1);
+    float colsum = cs0 + cs1;
+    float tacc = ta0 + ta1;
+    if (grp == 1) sCs[r] = colsum;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) tacc += __shfl_xor_sync(0xFFFFFFFFu, tacc, off);
+    if (lane == 0) ctl->tau_part[warp - 4] = tacc;
+    asm volatile("bar.sync 1, 256;" ::: "memory");  // the two warpgroups
+    if (grp == 0) {
+      ws.colsum[h * S_pad + j] = colsum + sCs[r];
+      if (r == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += ctl->tau_part[w];
+        ws.taup[h * n_kb + kb] = t;
+      }
+    }
+  }
+
+  tg::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && ctl->abort_flag) tg::set_device_error(err, TG_DEVERR_TIMEOUT);
+  if (warp == 2) {
+    tg::tc_fence_after();
+    tg::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------ reduce
+// Blocks [0, nb_ds): ds for 256 keys each; blocks nb_ds + h: dgain[h]; the last block:
+// dtau.  Every sum runs in a fixed order.
+__global__ void __launch_bounds__(256) attn_bwd_reduce_kernel(Workspace ws, const float *__restrict__ key_scores,
+                                                              const float *__restrict__ gain, int64_t S,
+                                                              int64_t S_pad, int Hq, int nb_ds, float inv_sqrt_d,
+                                                              float *__restrict__ ds, float *__restrict__ dgain,
+                                                              float *__restrict__ dtau) {
+  tg::pdl_wait();
+  tg::pdl_trigger();
+  __shared__ float red[256];
+  const int b = static_cast<int>(blockIdx.x);
+  const int t = threadIdx.x;
+  if (b < nb_ds) {
+    const int64_t j = static_cast<int64_t>(b) * 256 + t;
+    if (j < S) {
+      float acc = 0.f;
+      for (int h = 0; h < Hq; ++h) acc = fmaf(gain[h], ws.colsum[h * S_pad + j], acc);
+      ds[j] = acc;
+    }
+    return;
+  }
+  const int h = b - nb_ds;  // h == Hq: the temperature
+  float acc = 0.f;
+  if (h < Hq) {
+    for (int64_t j = t; j < S; j += 256) acc = fmaf(key_scores[j], ws.colsum[h * S_pad + j], acc);
+  } else {
+    const int64_t n = static_cast<int64_t>(Hq) * (S_pad / kBK);
+    for (int64_t i = t; i < n; i += 256) acc += ws.taup[i];
+  }
+  red[t] = acc;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (t < w) red[t] += red[t + w];
+    __syncthreads();
+  }
+  if (t == 0) {
+    if (h < Hq)
+      dgain[h] = red[0];
+    else
+      dtau[0] = red[0] * inv_sqrt_d;
+  }
+}
+
+bool tmap3(CUtensorMap *m, const void *base, int D, int heads, int64_t rows) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(heads), static_cast<uint64_t>(rows)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(heads) * D * 2};
+  const uint32_t box[3] = {64, 1, 128};
+  return tg::encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int D>
+tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain,
+                     float tau, const tg_bf16 *O, const float *O32, const tg_bf16 *dO, const float *lse, int64_t S,
+                     int32_t Hq, int32_t Hkv, const Workspace &ws, cudaStream_t stream, uint32_t *err) {
+  using C = BwdCfg<D>;
+  const int64_t S_pad = padded_rows(S);
+  const int n_kb = static_cast<int>(S_pad / kBK);
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  if (!tmap3(&tm_q, Q, D, Hq, S) || !tmap3(&tm_k, Kc, D, Hkv, S) || !tmap3(&tm_v, V, D, Hkv, S) ||
+      !tmap3(&tm_do, dO, D, Hq, S))
+    return TG_ERR_CUDA;
+  static bool configured[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::kSmem));
+    if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    // the warpgroup register split in the kernel assumes 168 registers per thread at launch
+    cudaFuncAttributes fa;
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, attn_bwd_kernel<D>);
+    if (ea != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(ea));
+    if (fa.numRegs != 168)
+      return tg::fail(TG_ERR_UNSUPPORTED, "attn_bwd_kernel built with %d registers per thread; the register split "
+                      "needs 168", fa.numRegs);
+    configured[dev] = true;
+  }
+  const int64_t prep_warps = S_pad * Hq;
+  const unsigned prep_grid = static_cast<unsigned>(std::min<int64_t>((prep_warps + 7) / 8, 8LL * tg::sm_count()));
+  cudaError_t e = tg::launch_pdl(attn_bwd_prep_kernel<D>, dim3(prep_grid), dim3(256), 0, stream,
+                                 reinterpret_cast<const __nv_bfloat16 *>(O), O32,
+                                 reinterpret_cast<const __nv_bfloat16 *>(dO), lse, S, S_pad, static_cast<int>(Hq), ws);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "attn_bwd_prep_kernel launch: %s", cudaGetErrorString(e));
+  const float c_log2 = tau / std::sqrt(static_cast<float>(D)) * kLog2e;
+  e = tg::launch_pdl(attn_bwd_kernel<D>, dim3(static_cast<unsigned>(n_kb * Hq)), dim3(kThreads), C::kSmem, stream, tm_q,
+                     tm_k, tm_v, tm_do, s, gain, c_log2, S, S_pad, static_cast<int>(Hq), static_cast<int>(Hkv), ws, err);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "attn_bwd_kernel launch: %s", cudaGetErrorString(e));
+  return TG_OK;
+}
+
+tg_status launch_reduce(const Workspace &ws, const float *s, const float *gain, int64_t S, int32_t Hq, int32_t D,
+                        float *ds, float *dgain, float *dtau, cudaStream_t stream) {
+  const int nb_ds = static_cast<int>((S + 255) / 256);
+  const cudaError_t e =
+      tg::launch_pdl(attn_bwd_reduce_kernel, dim3(static_cast<unsigned>(nb_ds + Hq + 1)), dim3(256), 0, stream, ws, s,
+                     gain, S, padded_rows(S), static_cast<int>(Hq), nb_ds, 1.0f / std::sqrt(static_cast<float>(D)), ds,
+                     dgain, dtau);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "attn_bwd_reduce_kernel launch: %s", cudaGetErrorString(e));
+  return TG_OK;
+}
+
+}  // namespace
+
+extern "C" size_t tg_gated_attention_backward_workspace(int64_t S, int32_t Hq) {
+  if (S < 0 || Hq <= 0) return 0;
+  return workspace_bytes(S, Hq);
+}
+
+extern "C" tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                                 const float *s, const float *gain, float tau, const tg_bf16 *O,
+                                                 const float *O32, const tg_bf16 *dO, const float *lse, int64_t S,
+                                                 int32_t Hq,
+                                                 int32_t Hkv, int32_t D, float *ds, float *dgain, float *dtau,
+                                                 void *workspace, size_t workspace_size, tg_stream stream) {
+  tg::clear_detail();
+  if (S < 0) return tg::fail(TG_ERR_INVALID_ARG, "S must be >= 0");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return tg::fail(TG_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv");
+  if (D != 64 && D != 128) return tg::fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+  if (!std::isfinite(tau)) return tg::fail(TG_ERR_INVALID_ARG, "tau must be finite");
+  if (padded_rows(S) * Hq > (int64_t(1) << 31) - 1) return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
+  if (!gain || !dgain || !dtau) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (S > 0 && (!Q || !Kc || !V || !s || (!O && !O32) || !dO || !lse || !ds || !workspace))
+    return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  const size_t need = workspace_bytes(S, Hq);
+  if (S > 0 && workspace_size < need)
+    return tg::fail(TG_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu bytes needed", workspace_size, need);
+  if (S > 0 && (!tg::aligned16(Q) || !tg::aligned16(Kc) || !tg::aligned16(V) || !tg::aligned16(dO) ||
+                !tg::aligned16(O) || !tg::aligned16(O32) || !tg::aligned16(workspace)))
+    return tg::fail(TG_ERR_ALIGNMENT, "Q, Kc, V, O, O32, dO and workspace must be 16-byte aligned");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Workspace ws = S > 0 ? carve(workspace, S, Hq) : Workspace{nullptr, nullptr, nullptr, nullptr};
+  if (S > 0) {
+    const tg_status r = D == 64 ? launch_bwd<64>(Q, Kc, V, s, gain, tau, O, O32, dO, lse, S, Hq, Hkv, ws, st, err)
+                                : launch_bwd<128>(Q, Kc, V, s, gain, tau, O, O32, dO, lse, S, Hq, Hkv, ws, st, err);
+    if (r != TG_OK) return r;
+  }
+  const tg_status r = launch_reduce(ws, s, gain, S, Hq, D, ds, dgain, dtau, st);
+  if (r != TG_OK) return r;
+  return tg::check_launch("tg_gated_attention_backward");
+}

@@ -375,6 +375,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 // acc0 += low bf16 of ``pair``, acc1 += high bf16 of ``pair`` (fp32 accumulation of bf16
 // operands, one mixed-precision add each).
 __device__ __forceinline__ void add_bf16x2_to_f32(float &acc0, float &acc1, uint32_t pair) {

@@ -8,6 +8,7 @@
     python -m learned_token_pruning_mlp_b200.runone gather --n 131072 --rows 8704
     python -m learned_token_pruning_mlp_b200.runone qkv --S 8704        # QKV + norm + rotary
     python -m learned_token_pruning_mlp_b200.runone oproj --S 8704      # output projection + residual
+    python -m learned_token_pruning_mlp_b200.runone attnbwd --S 8704    # backward w.r.t. s, gain, tau
 
 Each call is timed with CUDA events on the launching stream (after one warm-up
 call) and the mean per-call time is printed.  Shapes default to the 128k-context
@@ -27,7 +28,7 @@ from . import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention", "qkv", "oproj"])
+    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention", "qkv", "oproj", "attnbwd"])
     ap.add_argument("--n", type=int, default=131072)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--h", type=int, default=256)
@@ -96,6 +97,19 @@ def main():
         res = torch.randn(a.S, a.d, generator=g).to(torch.bfloat16).to(dev)
         y = torch.empty(a.S, a.d, dtype=torch.bfloat16, device=dev)
         fn = lambda: tg.tg_linear(x, Wo, res, y=y)
+    elif a.call == "attnbwd":
+        Q = torch.randn(a.S, a.hq, a.D, generator=g).to(torch.bfloat16).to(dev)
+        K = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
+        V = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
+        dO = torch.randn(a.S, a.hq, a.D, generator=g).to(torch.bfloat16).to(dev)
+        s = torch.randn(a.S, generator=g).to(dev)
+        gain = (0.5 + torch.rand(a.hq, generator=g)).to(dev)
+        O, lse, O32 = tg.tg_gated_attention_train(Q, K, V, s, gain, a.tau)
+        ds = torch.empty(a.S, device=dev)
+        dg = torch.empty(a.hq, device=dev)
+        dt = torch.empty(1, device=dev)
+        ws = torch.empty(tg.tg_gated_attention_backward_workspace(a.S, a.hq), dtype=torch.uint8, device=dev)
+        fn = lambda: tg.tg_gated_attention_backward(Q, K, V, s, gain, a.tau, O, dO, lse, O32, ds, dg, dt, workspace=ws)
     else:
         Q = torch.randn(a.S, a.hq, a.D, generator=g).to(torch.bfloat16).to(dev)
         K = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
@@ -131,7 +145,7 @@ def main():
     ms = e0.elapsed_time(e1) / a.repeat
     bits = tg.tg_get_device_error()
     extra = ""
-    if a.call == "attention":
+    if a.call in ("attention", "attnbwd"):
         fl = 4 * a.D * a.hq * a.S * (a.S + 1) / 2
         extra = f" {fl / ms / 1e9:.1f} TFLOP/s"
     elif a.call in ("qkv", "oproj"):

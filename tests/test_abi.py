@@ -118,6 +118,28 @@ def test_projections_reject_bad_arguments(L):
     assert L.tg_qkv_rope(p, 10, 64, p, p, b, None, None, f, 4, 2, 64, ctypes.c_void_p(4097), p, p, None) == 3
 
 
+def test_backward_workspace_size_and_argument_checks(L):
+    L.tg_gated_attention_backward_workspace.restype = ctypes.c_size_t
+    assert L.tg_gated_attention_backward_workspace(1000, 16) == 4 * 16 * (3 * 1024 + 8)   # padded to 1024 rows
+    assert L.tg_gated_attention_backward_workspace(1, 1) == 1792                            # 385 floats, 256-byte multiple
+    assert L.tg_gated_attention_backward_workspace(-1, 16) == 0
+    p = ctypes.c_void_p(4096)
+    f = ctypes.c_float(1.0)
+    big = ctypes.c_size_t(1 << 30)
+    args = lambda S, Hq, Hkv, D, ws=p, n=big, tau=f: (p, p, p, p, p, tau, p, None, p, p, S, Hq, Hkv, D, p, p, p, ws, n,  # noqa: E731
+                                                      None)
+    assert L.tg_gated_attention_backward(*args(100, 6, 4, 128)) == 1                       # Hq % Hkv
+    assert L.tg_gated_attention_backward(*args(100, 4, 2, 96)) == 2                        # D
+    assert L.tg_gated_attention_backward(*args(-1, 4, 2, 64)) == 1
+    assert L.tg_gated_attention_backward(*args(100, 4, 2, 64, tau=ctypes.c_float(float("nan")))) == 1
+    assert L.tg_gated_attention_backward(*args(100, 4, 2, 64, n=ctypes.c_size_t(1000))) == 1   # workspace too small
+    assert "workspace" in _detail(L)
+    assert L.tg_gated_attention_backward(*args(100, 4, 2, 64, ws=None)) == 1
+    assert L.tg_gated_attention_backward(*args(100, 4, 2, 64, ws=ctypes.c_void_p(4100))) == 3
+    assert L.tg_gated_attention_train(p, p, p, p, p, f, 10, 4, 2, 64, p, None, None, None) == 1   # lse NULL
+    assert L.tg_gated_attention_train(p, p, p, p, p, f, 10, 4, 2, 64, p, p, ctypes.c_void_p(4104), None) == 3
+
+
 def test_probe_rejects_bad_limit(L):
     assert L.tg_probe_wait_timeout(0, None) == 1
     assert L.tg_probe_wait_timeout(3_000_000_000, None) == 1
