@@ -10,6 +10,9 @@ whole step (27 layers of 4*D*Hq*S*(S+1)/2 flops divided by the full step time, t
 gate/top-K/gather time included); the gate+top-K+gather path is reported beside
 it in GB/s against HBM.  Inputs are resident in HBM before timing starts; the
 per-step working set (512 MiB residual + 1.9 GB of Q/K/V) is larger than L2.
+``next_rows`` gives the device time of the calls around the path on the same
+workload, outside the timed step: the pruned layer's projections, the attention
+backward, random-K and a 4-budget sweep.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {tokengate,reference}]
 """
@@ -38,7 +41,7 @@ DATASHEET_HBM_GBS = 8000.0
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch at
 # S = 8704, from the ncu capture summarised in profiles/attention_qwen3_1p7b_n128k_layer.md.
 # It is reported only while the kernel sources are the ones that capture measured.
-ATTENTION_TRAFFIC = {"sources_sha1": "bd210e913c3f163fade1ed41c4a9285cfc7dfd3c", "bytes_per_launch": 71461632 + 8472320}
+ATTENTION_TRAFFIC = {"sources_sha1": "d1e9b54d51050cb2b467c7c511a6eb7a7c90c52a", "bytes_per_launch": 71435008 + 8543232}
 
 
 def attention_traffic():
@@ -288,6 +291,7 @@ def run_tokengate(args, world, rank, local):
     # end to end through the public calls with host buffers: H2D of the step's inputs
     # from pinned memory and D2H of its results inside the timed region
     e2e = run_e2e(tg, host, dev, w, K, S, tau, world, args)
+    next_rows = time_next_rows(tg, dev, w, host, dv, kept, S)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -310,11 +314,77 @@ def run_tokengate(args, world, rank, local):
                      "traffic": attention_traffic(), "kernel": "gated_attention_kernel<128>",
                      "peak_source": f"{peaks['source']} bf16 sustained (kernel timed inside a long step)"},
         "e2e": e2e,
+        "next_rows": next_rows,
         "gpu_launches": args.steps * (3 + L),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(host, w, S, budget_s=args.cpu_seconds)
+    return out
+
+
+def time_next_rows(tg, dev, w, host, dv, kept, S, reps=5):
+    """Device time of the calls around the hot path on the same workload, outside the timed
+    step: the pruned layer's projections, the attention backward (training forward + backward),
+    random-K and a 4-budget sweep.  CUDA events on the launching stream, after one warm-up."""
+    from learned_token_pruning_mlp_b200 import workloads as W
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    Wq, Wo, qn, kn = (t.to(dev) for t in W.layer_weights(w))
+    Q, Kc, V = host["layers"][0]
+    Q, Kc, V = Q.to(dev), Kc.to(dev), V.to(dev)
+    s_k = torch.randn(S, generator=torch.Generator().manual_seed(5)).to(dev)
+    gain, tau = host["gain"].to(dev), host["tau"]
+    hk = torch.randn(S, w.d, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).to(dev)
+    pos = kept[:S].contiguous()
+    q_o = torch.empty_like(Q)
+    k_o, v_o = torch.empty_like(Kc), torch.empty_like(V)
+    y = torch.empty(S, w.d, dtype=torch.bfloat16, device=dev)
+    dO = torch.randn(S, w.hq, w.head_dim, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16).to(dev)
+    O, lse, O32 = tg.tg_gated_attention_train(Q, Kc, V, s_k, gain, tau)
+    ds = torch.empty(S, device=dev)
+    dg = torch.empty(w.hq, device=dev)
+    dt = torch.empty(1, device=dev)
+    ws = torch.empty(tg.tg_gated_attention_backward_workspace(S, w.hq), dtype=torch.uint8, device=dev)
+    kr = torch.empty(w.n, dtype=torch.int32, device=dev)
+    nkr = torch.empty(1, dtype=torch.int32, device=dev)
+    ks = torch.tensor([2048, 4096, 8192, 16384], dtype=torch.int32, device=dev)
+    ksw = torch.empty(4 * w.n, dtype=torch.int32, device=dev)
+    nksw = torch.empty(4, dtype=torch.int32, device=dev)
+    K = S - w.segments[0].q
+    D, hq, hkv, d = w.head_dim, w.hq, w.hkv, w.d
+    calls = {
+        "qkv_rope": (lambda: tg.tg_qkv_rope(hk, Wq, pos, w.rope_base, hq, hkv, D, qn, kn, w.norm_eps,
+                                            Q=q_o, Kc=k_o, V=v_o), 2 * S * (hq + 2 * hkv) * D * d, "tensor"),
+        "o_proj_residual": (lambda: tg.tg_linear(O.view(S, hq * D), Wo, hk, y=y), 2 * S * d * hq * D, "tensor"),
+        "attention_train_forward": (lambda: tg.tg_gated_attention_train(Q, Kc, V, s_k, gain, tau, O=O, lse=lse,
+                                                                         O32=O32), attention_flops(S, hq, D), "tensor"),
+        "attention_backward": (lambda: tg.tg_gated_attention_backward(Q, Kc, V, s_k, gain, tau, O, dO, lse, O32, ds,
+                                                                      dg, dt, workspace=ws),
+                               attention_flops(S, hq, D), "tensor"),
+        "random_k": (lambda: tg.tg_select_random_k(dv["mask"], K, 42, kept_idx=kr, n_kept=nkr), w.n + S * 4, "latency"),
+        "budget_sweep_4": (lambda: tg.tg_select_topk_sweep(dv["sel"], dv["mask"], ks, kept_idx=ksw, n_kept=nksw,
+                                                           stride=w.n), w.n * 5, "latency"),
+    }
+    out = {}
+    for name, (fn, work, bound) in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / reps * 1e3
+        row = {"us": round(us, 2), "reps": reps}
+        if bound == "tensor":
+            tf = work / (us * 1e-6) / 1e12
+            row.update({"tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)})
+        out[name] = row
+    bits = tg.tg_get_device_error()
+    if bits:
+        raise RuntimeError(f"device status bits {bits} after the next-row timings")
     return out
 
 
