@@ -263,6 +263,21 @@ tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16 *Kc, const
                                       float *ds, float *dgain, float *dtau,
                                       void *workspace, size_t workspace_bytes, tg_stream stream);
 
+/* tg_gated_attention_backward_noalloc -- the same backward without a caller
+ * workspace and without allocating anything: its scratch is a fixed 4 MiB device
+ * array inside the library (one per device), so any S * Hq whose workspace
+ * (tg_gated_attention_backward_workspace) exceeds 4,194,304 bytes is rejected
+ * with TG_ERR_UNSUPPORTED before any launch.  Calls on one device share that
+ * array: they must be ordered (one stream, or streams that wait on each other).
+ * Results are bitwise those of tg_gated_attention_backward.  The TokenGate article
+ * has no counterpart of this call: it is a deployment convenience of this library. */
+tg_status tg_gated_attention_backward_noalloc(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                              const float *s, const float *gain, float tau,
+                                              const tg_bf16 *O, const float *O32, const tg_bf16 *dO,
+                                              const float *lse, int64_t S, int32_t Hq, int32_t Hkv,
+                                              int32_t D, float *ds, float *dgain, float *dtau,
+                                              tg_stream stream);
+
 /* --------------------------------------------------------------------------
  * tg_qkv_rope -- Q, K and V of a pruned layer, at the kept tokens' positions.
  * TokenGate article, "How does TokenGate learned token pruning work?" (pruned

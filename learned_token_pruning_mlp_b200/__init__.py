@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     tg_gate_score,
     tg_gated_attention,
     tg_gated_attention_backward,
+    tg_gated_attention_backward_noalloc,
     tg_gated_attention_backward_workspace,
     tg_gated_attention_train,
     tg_gated_attention_varlen,

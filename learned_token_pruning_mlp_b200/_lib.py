@@ -57,6 +57,8 @@ _SIGNATURES = {
     "tg_gated_attention_backward_workspace": ([_i64, _i32], ctypes.c_size_t),
     "tg_gated_attention_backward": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp,
                                      _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
+    "tg_gated_attention_backward_noalloc": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i64, _i32, _i32,
+                                             _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
     "tg_qkv_rope": ([_vp, _i64, _i32, _vp, _vp, ctypes.c_double, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
                     ctypes.c_int),
     "tg_linear": ([_vp, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
@@ -280,6 +282,26 @@ def tg_gated_attention_varlen(Q, Kc, V, s, gain, tau: float, cu_seqlens, max_seq
         _dev(gain, torch.float32, "gain"), float(tau), _dev(cu_seqlens, torch.int32, "cu_seqlens"), B, total,
         int(max_seqlen), Hq, Hkv, D, _dev(O, bf, "O"), _stream(stream)))
     return O
+
+
+def tg_gated_attention_backward_noalloc(Q, Kc, V, s, gain, tau: float, O, dO, lse, O32=None, ds=None, dgain=None,
+                                        dtau=None, stream=None):
+    S, Hq, D = Q.shape
+    Hkv = Kc.shape[1]
+    dev = gain.device
+    if ds is None:
+        ds = torch.empty(S, dtype=torch.float32, device=dev)
+    if dgain is None:
+        dgain = torch.empty(Hq, dtype=torch.float32, device=dev)
+    if dtau is None:
+        dtau = torch.empty(1, dtype=torch.float32, device=dev)
+    bf = torch.bfloat16
+    _check("tg_gated_attention_backward_noalloc", lib().tg_gated_attention_backward_noalloc(
+        _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _dev(s, torch.float32, "s"),
+        _dev(gain, torch.float32, "gain"), float(tau), _dev(O, bf, "O"), _dev(O32, torch.float32, "O32"),
+        _dev(dO, bf, "dO"), _dev(lse, torch.float32, "lse"), S, Hq, Hkv, D, _dev(ds, torch.float32, "ds"),
+        _dev(dgain, torch.float32, "dgain"), _dev(dtau, torch.float32, "dtau"), _stream(stream)))
+    return ds, dgain, dtau
 
 
 def tg_qkv_rope(hidden, W_qkv, positions, rope_base: float, Hq: int, Hkv: int, D: int, q_norm=None, k_norm=None,

@@ -437,6 +437,12 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
   return TG_OK;
 }
 
+// Scratch of the allocation-free entry point: a fixed device array in this module's
+// global memory, 4 MiB (enough for S * Hq up to about 349,000 padded rows, e.g. the
+// 128k workload's layer, S = 8704 with 16 heads, which needs 1.7 MB).
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
+
 tg_status launch_reduce(const Workspace &ws, const float *s, const float *gain, int64_t S, int32_t Hq, int32_t D,
                         float *ds, float *dgain, float *dtau, cudaStream_t stream) {
   const int nb_ds = static_cast<int>((S + 255) / 256);
@@ -488,4 +494,40 @@ extern "C" tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16
   const tg_status r = launch_reduce(ws, s, gain, S, Hq, D, ds, dgain, dtau, st);
   if (r != TG_OK) return r;
   return tg::check_launch("tg_gated_attention_backward");
+}
+
+extern "C" tg_status tg_gated_attention_backward_noalloc(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                                         const float *s, const float *gain, float tau,
+                                                         const tg_bf16 *O, const float *O32, const tg_bf16 *dO,
+                                                         const float *lse, int64_t S, int32_t Hq, int32_t Hkv,
+                                                         int32_t D, float *ds, float *dgain, float *dtau,
+                                                         tg_stream stream) {
+  tg::clear_detail();
+  if (S < 0) return tg::fail(TG_ERR_INVALID_ARG, "S must be >= 0");
+  if (Hq <= 0) return tg::fail(TG_ERR_INVALID_ARG, "Hq must be positive");
+  if (padded_rows(S) * Hq > (int64_t(1) << 31) - 1) return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
+  const size_t need = workspace_bytes(S, Hq);
+  if (need > kStaticScratchBytes)
+    return tg::fail(TG_ERR_UNSUPPORTED,
+                    "S = %lld with Hq = %d needs %zu bytes of scratch; the static scratch of this entry point holds "
+                    "%zu bytes (use tg_gated_attention_backward with a caller workspace)",
+                    static_cast<long long>(S), Hq, need, kStaticScratchBytes);
+  void *scratch = nullptr;
+  if (S > 0) {
+    // the array's address on the current device, looked up once per device
+    static void *cached[64];
+    int dev = 0;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(ed));
+    if (dev >= 0 && dev < 64 && cached[dev]) {
+      scratch = cached[dev];
+    } else {
+      const cudaError_t e = cudaGetSymbolAddress(&scratch, g_bwd_scratch);
+      if (e != cudaSuccess || !scratch)
+        return tg::fail(TG_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+      if (dev >= 0 && dev < 64) cached[dev] = scratch;
+    }
+  }
+  return tg_gated_attention_backward(Q, Kc, V, s, gain, tau, O, O32, dO, lse, S, Hq, Hkv, D, ds, dgain, dtau, scratch,
+                                     kStaticScratchBytes, stream);
 }

@@ -140,6 +140,16 @@ def test_backward_workspace_size_and_argument_checks(L):
     assert L.tg_gated_attention_train(p, p, p, p, p, f, 10, 4, 2, 64, p, p, ctypes.c_void_p(4104), None) == 3
 
 
+def test_backward_noalloc_rejects_sizes_beyond_its_static_scratch(L):
+    p = ctypes.c_void_p(4096)
+    f = ctypes.c_float(1.0)
+    # S = 30000 with 16 heads needs 4 * 16 * (3 * 30080 + 235) bytes > 4 MiB: rejected before any CUDA call
+    assert L.tg_gated_attention_backward_noalloc(p, p, p, p, p, f, p, None, p, p, 30000, 16, 8, 128,
+                                                 p, p, p, None) == 2
+    assert "static scratch" in _detail(L) and "4194304" in _detail(L)
+    assert L.tg_gated_attention_backward_noalloc(p, p, p, p, p, f, p, None, p, p, -1, 16, 8, 128, p, p, p, None) == 1
+
+
 def test_probe_rejects_bad_limit(L):
     assert L.tg_probe_wait_timeout(0, None) == 1
     assert L.tg_probe_wait_timeout(3_000_000_000, None) == 1
