@@ -167,6 +167,34 @@ tg_status tg_select_random_k(const uint8_t *doc_mask, int64_t n, int64_t k, uint
                              int32_t *kept_idx, int64_t cap, int32_t *n_kept, tg_stream stream);
 
 /* --------------------------------------------------------------------------
+ * tg_select_fused -- tg_gate_score, tg_select_topk and tg_gather as one call.
+ * TokenGate article, "How does TokenGate learned token pruning work?": the gate
+ * scores every token, the K best document tokens and every question token are
+ * kept, and the layers above L run on the kept tokens only.  The results are
+ * exactly those of the three calls in sequence on the same arguments:
+ *     scores  = tg_gate_score(hidden, W1, b1, W2, b2)                fp32 [n]
+ *     kept_idx, *n_kept = tg_select_topk(scores, doc_mask, k, cap)
+ *     hidden_k, s_k = tg_gather(hidden, kept_idx, n_rows, n_kept, scores)
+ * Faster: the gate's epilogue histograms the top byte of every document token's
+ * selection key, so the selector's first radix pass reads those histograms
+ * instead of every score, and the three kernels overlap at their boundaries.
+ *   workspace: device memory of at least tg_select_fused_workspace(n) bytes
+ *   (depends on the current device's SM count), 16-byte aligned, caller-owned;
+ *   it holds the per-CTA histograms until the stream reaches the end of the call.
+ * Sizes as for the three calls (d a multiple of 8, at most 16384; h a multiple of
+ * 16 in [16, 256]; n < 2^31); n_rows <= cap; hidden_k and s_k are required when
+ * n_rows > 0.  Device-side conditions set the same status bits as the three calls.
+ * -------------------------------------------------------------------------- */
+size_t tg_select_fused_workspace(int64_t n);
+
+tg_status tg_select_fused(const tg_bf16 *hidden, int64_t n, int32_t d, const tg_bf16 *W1,
+                          const tg_bf16 *b1, const tg_bf16 *W2, const tg_bf16 *b2, int32_t h,
+                          const uint8_t *doc_mask, int64_t k, float *scores, int32_t *kept_idx,
+                          int64_t cap, int32_t *n_kept, tg_bf16 *hidden_k, float *s_k,
+                          int64_t n_rows, void *workspace, size_t workspace_bytes,
+                          tg_stream stream);
+
+/* --------------------------------------------------------------------------
  * tg_gather -- compaction of the kept tokens.
  * TokenGate article, "How does TokenGate learned token pruning work?" (pruned
  * forward): layers above the gate process only the kept tokens and create no

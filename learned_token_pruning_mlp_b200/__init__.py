@@ -30,6 +30,8 @@ from ._lib import (  # noqa: F401
     tg_linear,
     tg_probe_wait_timeout,
     tg_qkv_rope,
+    tg_select_fused,
+    tg_select_fused_workspace,
     tg_select_random_k,
     tg_select_topk,
     tg_select_topk_sweep,

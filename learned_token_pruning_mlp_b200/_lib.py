@@ -48,6 +48,9 @@ _SIGNATURES = {
     "tg_select_topk_varlen": ([_vp, _vp, _vp, _i32, _i64, _vp, _i64, _vp, _i64, _vp, _vp], ctypes.c_int),
     "tg_select_topk_sweep": ([_vp, _vp, _i64, _vp, _i32, _vp, _i64, _vp, _vp], ctypes.c_int),
     "tg_select_random_k": ([_vp, _i64, _i64, ctypes.c_uint64, _vp, _i64, _vp, _vp], ctypes.c_int),
+    "tg_select_fused_workspace": ([_i64], ctypes.c_size_t),
+    "tg_select_fused": ([_vp, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp,
+                         ctypes.c_size_t, _vp], ctypes.c_int),
     "tg_gather": ([_vp, _i64, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "tg_gated_attention": ([_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp, _vp], ctypes.c_int),
     "tg_gated_attention_varlen": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp, _vp],
@@ -193,6 +196,42 @@ def tg_select_random_k(doc_mask, k: int, seed: int, kept_idx=None, n_kept=None, 
         _dev(doc_mask, torch.uint8, "doc_mask"), n, int(k), int(seed) & 0xFFFFFFFFFFFFFFFF,
         _dev(kept_idx, torch.int32, "kept_idx"), int(cap), _dev(n_kept, torch.int32, "n_kept"), _stream(stream)))
     return kept_idx, n_kept
+
+
+def tg_select_fused_workspace(n: int) -> int:
+    return int(lib().tg_select_fused_workspace(int(n)))
+
+
+def tg_select_fused(hidden, W1, b1, W2, b2, doc_mask, k: int, n_rows: Optional[int] = None, scores=None,
+                    kept_idx=None, n_kept=None, hidden_k=None, s_k=None, cap: Optional[int] = None, workspace=None,
+                    stream=None):
+    """Gate -> top-K -> gather in one call; returns (scores, kept_idx, n_kept, hidden_k, s_k)."""
+    n, d = hidden.shape
+    h = W1.shape[0]
+    dev = hidden.device
+    if scores is None:
+        scores = torch.empty(n, dtype=torch.float32, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(max(n, 1), dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.empty(1, dtype=torch.int32, device=dev)
+    cap = kept_idx.numel() if cap is None else cap
+    if n_rows is None:
+        n_rows = min(cap, n)
+    if hidden_k is None:
+        hidden_k = torch.empty((max(n_rows, 1), d), dtype=hidden.dtype, device=dev)
+    if s_k is None:
+        s_k = torch.empty(max(n_rows, 1), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(tg_select_fused_workspace(n), 16), dtype=torch.uint8, device=dev)
+    bf = torch.bfloat16
+    _check("tg_select_fused", lib().tg_select_fused(
+        _dev(hidden, bf, "hidden"), n, d, _dev(W1, bf, "W1"), _dev(b1, bf, "b1"), _dev(W2, bf, "W2"),
+        _dev(b2, bf, "b2"), h, _dev(doc_mask, torch.uint8, "doc_mask"), int(k), _dev(scores, torch.float32, "scores"),
+        _dev(kept_idx, torch.int32, "kept_idx"), int(cap), _dev(n_kept, torch.int32, "n_kept"),
+        _dev(hidden_k, bf, "hidden_k"), _dev(s_k, torch.float32, "s_k"), int(n_rows),
+        _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)))
+    return scores, kept_idx, n_kept, hidden_k, s_k
 
 
 def tg_gather(hidden, kept_idx, n_rows: Optional[int] = None, n_kept=None, hidden_k=None, scores=None, s_k=None,

@@ -66,10 +66,13 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
             for (src, _), log in zip(jobs, ex.map(lambda j: _compile(j[0], j[1], ptxas_verbose), jobs)):
                 if ptxas_verbose or (log.strip() and not quiet):
                     print(f"== {os.path.basename(src)}\n{log}", file=sys.stderr)
+    export_map = os.path.join(CSRC, "exports.map")
     if jobs or force or not os.path.exists(LIB) or \
-            os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
+            os.path.getmtime(LIB) < max(max(os.path.getmtime(o) for o in objs), os.path.getmtime(export_map)):
         tmp = LIB + f".tmp{os.getpid()}"
-        r = subprocess.run([nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp],
+        # export the C ABI only (csrc/exports.map)
+        r = subprocess.run([nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC",
+                            f"-Xlinker=--version-script={os.path.join(CSRC, 'exports.map')}", *objs, "-o", tmp],
                            capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -25,10 +25,16 @@
 //     one fp32 per token.  The hidden activations never leave the SM.
 // The residual is streamed with an L2 evict-first hint and W1 (re-read by every
 // tile) with evict-last, so W1 stays L2-resident while the residual passes through.
+// For the fused selection (tg_select_fused) the epilogue also histograms the top 8
+// bits of the selector's order key of each document token's score (warp-aggregated
+// shared-memory atomics) and every CTA stores its 256 bins: the selector's first
+// radix pass then sums those instead of reading the scores.
 #include <algorithm>
 
+#include "internal.h"
 #include "ptx.cuh"
 #include "runtime.h"
+#include "select_key.cuh"
 
 namespace {
 
@@ -49,6 +55,7 @@ struct GateCtl {
   int abort_flag;
   float b1[kMaxH];
   float w2[kMaxH];
+  uint32_t hist[256];          // top-byte histogram of the document tokens' order keys
 };
 
 constexpr size_t smem_bytes(int h) {
@@ -60,7 +67,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gate_score_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                       const __nv_bfloat16 *__restrict__ b1, const __nv_bfloat16 *__restrict__ W2,
                       const __nv_bfloat16 *__restrict__ b2, float *__restrict__ scores, int64_t n, int d, int h,
-                      uint32_t tmem_cols, uint32_t *err) {
+                      uint32_t tmem_cols, const uint8_t *__restrict__ doc_mask, uint32_t *__restrict__ hist_parts,
+                      uint32_t *err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -109,6 +117,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ctl->b1[j] = __bfloat162float(b1[j]);
       ctl->w2[j] = __bfloat162float(W2[j]);
     }
+    if (hist_parts)
+      for (int j = threadIdx.x - 128; j < 256; j += 128) ctl->hist[j] = 0;
     asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
   }
   const uint32_t tmem_base = ctl->tmem_base;
@@ -192,7 +202,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tg::tc_fence_before();
       tg::mbar_arrive_remote(tg::smem_addr(&ctl->acc_empty[acc]), 0u);  // the leader's copy
       const int64_t row = tile * 2 * kBlockM + rank * kBlockM + quarter * 32 + lane;
-      if (row < n) scores[row] = sum + bias2;
+      const float score = sum + bias2;
+      if (row < n) scores[row] = score;
+      if (hist_parts) {
+        // lanes with the same top byte add once, with the group's size
+        const uint32_t key = row < n ? tg::order_key(score, doc_mask[row] != 0) : 0u;
+        const unsigned live = __ballot_sync(0xFFFFFFFFu, key != 0u);
+        if (key != 0u) {
+          const unsigned peers = __match_any_sync(live, key >> 24);
+          if (lane == __ffs(peers) - 1) atomicAdd(&ctl->hist[key >> 24], static_cast<uint32_t>(__popc(peers)));
+        }
+      }
+    }
+    if (hist_parts) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // every epilogue warp has added its tiles
+      for (int j = threadIdx.x - 128; j < 256; j += 128) hist_parts[blockIdx.x * 256 + j] = ctl->hist[j];
     }
   }
 
@@ -209,15 +233,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, const tg_bf16 *W1, const tg_bf16 *b1,
-                                   const tg_bf16 *W2, const tg_bf16 *b2, int32_t h, float *scores, tg_stream stream) {
-  tg::clear_detail();
+int64_t tg::gate_grid(int64_t n) {
+  const int64_t num_tiles = (n + 2 * kBlockM - 1) / (2 * kBlockM);
+  return 2 * std::min<int64_t>(num_tiles, tg::sm_count() / 2);
+}
+
+tg_status tg::gate_score_hist(const tg_bf16 *hidden, int64_t n, int32_t d, const tg_bf16 *W1, const tg_bf16 *b1,
+                              const tg_bf16 *W2, const tg_bf16 *b2, int32_t h, float *scores, const uint8_t *doc_mask,
+                              uint32_t *hist_parts, tg_stream stream) {
   if (n < 0) return tg::fail(TG_ERR_INVALID_ARG, "n must be >= 0");
   if (d <= 0 || d % 8 != 0) return tg::fail(TG_ERR_INVALID_ARG, "d must be a positive multiple of 8 (got %d)", d);
   if (h < 16 || h > kMaxH || h % 16 != 0)
     return tg::fail(TG_ERR_UNSUPPORTED, "h must be a multiple of 16 in [16, 256] (got %d)", h);
   if (n == 0) return TG_OK;
   if (!hidden || !W1 || !b1 || !W2 || !b2 || !scores) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (hist_parts && !doc_mask) return tg::fail(TG_ERR_INVALID_ARG, "doc_mask is NULL");
   if (!tg::aligned16(hidden) || !tg::aligned16(W1) || !tg::aligned16(scores))
     return tg::fail(TG_ERR_ALIGNMENT, "hidden, W1 and scores must be 16-byte aligned");
   if (n > (int64_t(1) << 31) * kBlockM) return tg::fail(TG_ERR_UNSUPPORTED, "n too large");
@@ -254,13 +284,18 @@ extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, 
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     configured[dev] = true;
   }
-  const int64_t num_tiles = (n + 2 * kBlockM - 1) / (2 * kBlockM);
-  const int64_t pairs = std::min<int64_t>(num_tiles, tg::sm_count() / 2);
-  const cudaError_t e = tg::launch_pdl(gate_score_kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem,
+  const cudaError_t e = tg::launch_pdl(gate_score_kernel, dim3(static_cast<unsigned>(gate_grid(n))), dim3(kThreads), smem,
                                       static_cast<cudaStream_t>(stream), tm_x, tm_w,
                                       reinterpret_cast<const __nv_bfloat16 *>(b1),
                                       reinterpret_cast<const __nv_bfloat16 *>(W2),
-                                      reinterpret_cast<const __nv_bfloat16 *>(b2), scores, n, d, h, tmem_cols, err);
+                                      reinterpret_cast<const __nv_bfloat16 *>(b2), scores, n, d, h, tmem_cols, doc_mask,
+                                      hist_parts, err);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gate_score_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("gate_score_kernel");
+}
+
+extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, const tg_bf16 *W1, const tg_bf16 *b1,
+                                   const tg_bf16 *W2, const tg_bf16 *b2, int32_t h, float *scores, tg_stream stream) {
+  tg::clear_detail();
+  return tg::gate_score_hist(hidden, n, d, W1, b1, W2, b2, h, scores, nullptr, nullptr, stream);
 }

@@ -24,8 +24,10 @@
 
 #include <algorithm>
 
+#include "internal.h"
 #include "ptx.cuh"
 #include "runtime.h"
+#include "select_key.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -38,15 +40,7 @@ constexpr int kItems = 16;                        // consecutive positions per t
 constexpr int kRound = kThreads * kItems;         // positions per CTA per round (16384)
 constexpr int kBins = 256;                        // 8-bit digits, four passes at most
 
-// Order key: larger key = earlier in (score desc, NaN last).  0 marks a question
-// token (never competes), 1 is NaN, every number maps to >= 0x007FFFFF.
-__device__ __forceinline__ uint32_t order_key(float f, bool doc) {
-  if (!doc) return 0u;
-  uint32_t b = __float_as_uint(f);
-  if ((b & 0x7FFFFFFFu) > 0x7F800000u) return 1u;  // NaN
-  if (b == 0x80000000u) b = 0u;                      // -0.0 ranks with +0.0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
+using tg::order_key;
 
 struct TopkShared {
   uint32_t hist[2][kBins];     // double-buffered per-CTA histograms (read by the cluster)
@@ -153,6 +147,8 @@ struct TopkArgs {
   int32_t *n_kept;            // single: [1]; sweep: [number of budgets]
   uint64_t seed;              // random mode: key = SplitMix64(seed, position)
   int random;
+  const uint32_t *hist_parts; // single mode: n_parts histograms of the keys' top byte (pass 0)
+  int n_parts;
   uint32_t *err;
 };
 
@@ -282,11 +278,21 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       if (threadIdx.x < kBins) sh.hist[buf][threadIdx.x] = 0;
       __syncthreads();
     }
-    for (int rd = 0; rd < rounds; ++rd) {
-      if (!kResident) load_keys(rd);
+    if (pass == 0 && args.hist_parts) {
+      // the first digit's histogram was built by the producer of the scores: sum this
+      // CTA's share of its partial histograms (the cluster reduction adds the shares)
+      if (threadIdx.x < kBins) {
+        uint32_t c = 0;
+        for (int p = rank; p < args.n_parts; p += kCluster) c += __ldg(args.hist_parts + p * kBins + threadIdx.x);
+        sh.hist[0][threadIdx.x] = c;
+      }
+    } else {
+      for (int rd = 0; rd < rounds; ++rd) {
+        if (!kResident) load_keys(rd);
 #pragma unroll
-      for (int e = 0; e < kItems; ++e)
-        if (keys[e] != 0u && (keys[e] & pmask) == prefix) atomicAdd(&sh.hist[buf][(keys[e] >> shift) & 0xFFu], 1u);
+        for (int e = 0; e < kItems; ++e)
+          if (keys[e] != 0u && (keys[e] & pmask) == prefix) atomicAdd(&sh.hist[buf][(keys[e] >> shift) & 0xFFu], 1u);
+      }
     }
     __syncthreads();
     cluster.sync();
@@ -504,6 +510,35 @@ extern "C" tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask
   a.kept_idx = kept_idx;
   a.cap = cap;
   a.n_kept = n_kept;
+  a.err = err;
+  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
+  if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
+  return tg::check_launch("topk_cluster_kernel");
+}
+
+tg_status tg::select_topk_hist(const float *scores, const uint8_t *doc_mask, int64_t n, int64_t k, int32_t *kept_idx,
+                               int64_t cap, int32_t *n_kept, const uint32_t *hist_parts, int n_parts,
+                               tg_stream stream) {
+  if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
+  if (k < 0) return tg::fail(TG_ERR_INVALID_ARG, "k must be >= 0");
+  if (cap < 0) return tg::fail(TG_ERR_INVALID_ARG, "cap must be >= 0");
+  if (!n_kept) return tg::fail(TG_ERR_INVALID_ARG, "n_kept is NULL");
+  if (n > 0 && (!scores || !doc_mask)) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (cap > 0 && !kept_idx) return tg::fail(TG_ERR_INVALID_ARG, "kept_idx is NULL");
+  if (n > 0 && (!hist_parts || n_parts <= 0)) return tg::fail(TG_ERR_INVALID_ARG, "no first-pass histograms");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  TopkArgs a = {};
+  a.scores = scores;
+  a.mask = doc_mask;
+  a.n_single = n;
+  a.k_single = k;
+  a.total = n;
+  a.kept_idx = kept_idx;
+  a.cap = cap;
+  a.n_kept = n_kept;
+  a.hist_parts = hist_parts;
+  a.n_parts = n_parts;
   a.err = err;
   const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));

@@ -9,6 +9,8 @@
     python -m learned_token_pruning_mlp_b200.runone qkv --S 8704        # QKV + norm + rotary
     python -m learned_token_pruning_mlp_b200.runone oproj --S 8704      # output projection + residual
     python -m learned_token_pruning_mlp_b200.runone attnbwd --S 8704    # backward w.r.t. s, gain, tau
+    python -m learned_token_pruning_mlp_b200.runone fused --graph       # gate -> top-K -> gather, one call
+    python -m learned_token_pruning_mlp_b200.runone chain --graph       # the same as three calls
 
 Each call is timed with CUDA events on the launching stream (after one warm-up
 call) and the mean per-call time is printed.  Shapes default to the 128k-context
@@ -28,7 +30,7 @@ from . import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention", "qkv", "oproj", "attnbwd"])
+    ap.add_argument("call", choices=["gate", "topk", "randomk", "sweep", "gather", "attention", "qkv", "oproj", "attnbwd", "fused", "chain"])
     ap.add_argument("--n", type=int, default=131072)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--h", type=int, default=256)
@@ -97,6 +99,29 @@ def main():
         res = torch.randn(a.S, a.d, generator=g).to(torch.bfloat16).to(dev)
         y = torch.empty(a.S, a.d, dtype=torch.bfloat16, device=dev)
         fn = lambda: tg.tg_linear(x, Wo, res, y=y)
+    elif a.call in ("fused", "chain"):
+        hidden = torch.randn(a.n, a.d, generator=g).to(torch.bfloat16).to(dev)
+        W1 = (torch.randn(a.h, a.d, generator=g) / math.sqrt(a.d)).to(torch.bfloat16).to(dev)
+        b1 = torch.zeros(a.h, dtype=torch.bfloat16, device=dev)
+        W2 = (torch.randn(a.h, generator=g) / math.sqrt(a.h)).to(torch.bfloat16).to(dev)
+        b2 = torch.zeros(1, dtype=torch.bfloat16, device=dev)
+        m = torch.ones(a.n, dtype=torch.uint8, device=dev)
+        m[-512:] = 0
+        S = a.k + 512
+        sc = torch.empty(a.n, dtype=torch.float32, device=dev)
+        kept = torch.empty(a.n, dtype=torch.int32, device=dev)
+        nk = torch.empty(1, dtype=torch.int32, device=dev)
+        hk = torch.empty(S, a.d, dtype=torch.bfloat16, device=dev)
+        sk = torch.empty(S, dtype=torch.float32, device=dev)
+        ws = torch.empty(tg.tg_select_fused_workspace(a.n), dtype=torch.uint8, device=dev)
+        if a.call == "fused":
+            fn = lambda: tg.tg_select_fused(hidden, W1, b1, W2, b2, m, a.k, n_rows=S, scores=sc, kept_idx=kept,
+                                            n_kept=nk, hidden_k=hk, s_k=sk, workspace=ws)
+        else:
+            def fn():
+                tg.tg_gate_score(hidden, W1, b1, W2, b2, scores=sc)
+                tg.tg_select_topk(sc, m, a.k, kept_idx=kept, n_kept=nk)
+                tg.tg_gather(hidden, kept, n_rows=S, n_kept=nk, hidden_k=hk, scores=sc, s_k=sk)
     elif a.call == "attnbwd":
         Q = torch.randn(a.S, a.hq, a.D, generator=g).to(torch.bfloat16).to(dev)
         K = torch.randn(a.S, a.hkv, a.D, generator=g).to(torch.bfloat16).to(dev)
@@ -148,6 +173,10 @@ def main():
     if a.call in ("attention", "attnbwd"):
         fl = 4 * a.D * a.hq * a.S * (a.S + 1) / 2
         extra = f" {fl / ms / 1e9:.1f} TFLOP/s"
+    elif a.call in ("fused", "chain"):
+        S = a.k + 512
+        by = a.n * a.d * 2 + a.h * a.d * 2 + a.n * 4 + a.n * 4 + a.n + S * 4 + 2 * S * a.d * 2 + 2 * S * 4
+        extra = f" {by / ms / 1e6:.1f} GB/s algorithmic"
     elif a.call in ("qkv", "oproj"):
         n_out = (a.hq + 2 * a.hkv) * a.D if a.call == "qkv" else a.d
         k_in = a.d if a.call == "qkv" else a.hq * a.D

@@ -38,6 +38,13 @@ def test_every_declared_symbol_is_exported(L):
     assert not missing, missing
 
 
+def test_library_exports_only_the_declared_calls(L):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    assert exported == set(_declared()), exported ^ set(_declared())
+
+
 def test_binding_covers_every_declared_symbol():
     assert set(_declared()) <= set(_lib._SIGNATURES)
 
@@ -148,6 +155,18 @@ def test_backward_noalloc_rejects_sizes_beyond_its_static_scratch(L):
                                                  p, p, p, None) == 2
     assert "static scratch" in _detail(L) and "4194304" in _detail(L)
     assert L.tg_gated_attention_backward_noalloc(p, p, p, p, p, f, p, None, p, p, -1, 16, 8, 128, p, p, p, None) == 1
+
+
+def test_select_fused_rejects_bad_arguments(L):
+    p = ctypes.c_void_p(4096)
+    ws = ctypes.c_size_t(1 << 20)
+    args = lambda n=1000, d=64, h=64, k=10, cap=100, rows=50, hk=p, sk=p: (  # noqa: E731
+        p, n, d, p, p, p, p, h, p, k, p, p, cap, p, hk, sk, rows, p, ws, None)
+    assert L.tg_select_fused(*args(n=-1)) == 1
+    assert L.tg_select_fused(*args(rows=101)) == 1          # n_rows > cap
+    assert L.tg_select_fused(*args(d=12)) == 2              # d % 8
+    assert L.tg_select_fused(*args(d=32768)) == 2           # d above the gather's limit
+    assert L.tg_select_fused(*args(hk=None)) == 1           # rows requested without hidden_k
 
 
 def test_probe_rejects_bad_limit(L):
