@@ -29,9 +29,10 @@
 //     be issued right after O_t += P_t(j) V_j even though it overwrites P_t(j).
 //   * warps 4-7 and 8-11 are the softmax warpgroups of tile 0 and tile 1 (one query
 //     row per thread): tcgen05.ld of the S' row, causal mask on the diagonal tile,
-//     8-way max, exp2 of one packed f32x2 FMA per pair, bf16 pack, 8-way sum of the
-//     rounded weights with mixed-precision adds (so normalisation matches the
-//     weights the PV product uses), tcgen05.st of P.  While one warpgroup works on its softmax the tensor core
+//     exp2 of one packed f32x2 FMA per pair against the running max with the tile's
+//     max taken in the same pass, bf16 pack, 8-way sum of the rounded weights with
+//     mixed-precision adds (so normalisation matches the weights the PV product
+//     uses), tcgen05.st of P.  While one warpgroup works on its softmax the tensor core
 //     works on the other tile's products.
 //   * The running max is only moved when it grows by more than 2^8 for some row of
 //     the warp (decided per warp: TMEM access is warp-collective); then O_t is
@@ -180,10 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Register split: the launch gives 384 threads x 168 registers; the loader/MMA
   // warpgroup needs few, the two softmax warpgroups hold a 128-wide S row each.
-  // 128 x 56 + 256 x 224 = 384 x 168, so the increase never waits.  Each warpgroup
-  // changes its budget inside its own branch.
+  // 128 x 64 + 256 x 216 = 63488 <= 384 x 168, so the increase never waits (the
+  // launcher checks the launch count).  Each warpgroup changes its budget inside its
+  // own branch.
   if (warp < 4) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
     const int nq = n1 ? 2 : 1;
@@ -232,30 +234,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, D, false, true);
     bool ok = tg::mbar_wait(tg::smem_addr(&ctl->q_full), 0, abort_flag);
 
+    // Shared-memory descriptors, built once: a descriptor is two 32-bit words, and the
+    // operand of each K step differs from its tile's by a constant offset added to the
+    // start-address field of the low word (16-byte units, 14 bits; shared addresses stay
+    // below 2^18 bytes, so the add never carries out of the field).  This keeps the
+    // issuing thread's instruction count per MMA low: it shares its SM sub-partition
+    // with two softmax warps.
+    const uint64_t dsw = tg::smem_desc_sw128(tg::smem_addr(sQ), 16, 1024);
+    const uint32_t hi_sw = static_cast<uint32_t>(dsw >> 32);
+    const uint32_t q_lo0 = static_cast<uint32_t>(dsw);
+    const uint32_t k_lo0 = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sK), 16, 1024));
+    const uint64_t dv = tg::smem_desc_sw128(tg::smem_addr(sV), kHalfBytes, 1024);
+    const uint32_t v_lo0 = static_cast<uint32_t>(dv), hi_v = static_cast<uint32_t>(dv >> 32);
+    const uint64_t dqx = tg::smem_desc_noswz(tg::smem_addr(sQx), kExtLBO, kExtSBO);
+    const uint64_t dkx = tg::smem_desc_noswz(tg::smem_addr(sKx), kExtLBO, kExtSBO);
+    const uint32_t kx_lo0 = static_cast<uint32_t>(dkx), hi_x = static_cast<uint32_t>(dkx >> 32);
+    constexpr uint32_t kTileUnits = C::kTileBytes >> 4;
+
     auto issue_s = [&](int t, int j) {
-      const int s = j % NS;
+      const uint32_t s = static_cast<uint32_t>(j % NS);
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(t * kBN);
-      tg::mma_bf16_ss(d_tmem, tg::smem_desc_noswz(tg::smem_addr(sQx), kExtLBO, kExtSBO),
-                      tg::smem_desc_noswz(tg::smem_addr(sKx + s * kExtBytes), kExtLBO, kExtSBO), idesc_s, 0u);
+      tg::mma_bf16_ss(d_tmem, dqx, tg::desc_words(kx_lo0 + s * (kExtBytes >> 4), hi_x), idesc_s, 0u);
       if (!skip_qk) {
+        const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(t) * kTileUnits, k_lo = k_lo0 + s * kTileUnits;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
-          const uint64_t ad = tg::smem_desc_sw128(tg::smem_addr(sQ + t * C::kTileBytes) + off, 16, 1024);
-          const uint64_t bd = tg::smem_desc_sw128(tg::smem_addr(sK + s * C::kTileBytes) + off, 16, 1024);
-          tg::mma_bf16_ss(d_tmem, ad, bd, idesc_s, 1u);
+          const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+          tg::mma_bf16_ss(d_tmem, tg::desc_words(q_lo + off, hi_sw), tg::desc_words(k_lo + off, hi_sw), idesc_s, 1u);
         }
       }
       tg::mma_commit(tg::smem_addr(&ctl->s_full[t]));
     };
     auto issue_pv = [&](int t, int j) {
-      const int s = j % NS;
+      const uint32_t s = static_cast<uint32_t>(j % NS);
       const uint32_t d_tmem = tmem_base + 256u + static_cast<uint32_t>(t * D);
       const uint32_t p_tmem = tmem_base + static_cast<uint32_t>(t * kBN);
+      const uint32_t v_lo = v_lo0 + s * kTileUnits;
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk) {
         // 16 keys = 16 rows of V (2 swizzle groups of 8 rows, 2048 bytes); D blocks 16 KB apart
-        const uint64_t bd = tg::smem_desc_sw128(tg::smem_addr(sV + s * C::kTileBytes) + kk * 2048u, kHalfBytes, 1024);
+        const uint64_t bd = tg::desc_words(v_lo + static_cast<uint32_t>(kk) * (2048u >> 4), hi_v);
         tg::mma_bf16_ts(d_tmem, p_tmem + kk * 8u, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
       }
     };
@@ -304,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
     // ------------------------------------------------------------ softmax + epilogue
     const int t = (warp - 4) >> 2;          // query tile of this warpgroup
     const int quarter = warp & 3;           // TMEM lane quarter
@@ -325,43 +343,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tg::tc_fence_after();
       uint32_t x[kBN];
+      // the S' row of this tile from TMEM, causal mask on the diagonal tile
+      auto load_row = [&]() {
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tg::tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
-      tg::tmem_ld_wait();
-      if (j == diag) {
+        for (int c = 0; c < kBN / 32; ++c) tg::tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
+        tg::tmem_ld_wait();
+        if (j == diag) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c > r) x[c] = __float_as_uint(-INFINITY);
-      }
-      float mx[8];
+          for (int c = 0; c < kBN; ++c)
+            if (c > r) x[c] = __float_as_uint(-INFINITY);
+        }
+      };
+      float acc[8], mx[8];
+      // exp2(eff S' - eff m) for the row, packed to bf16 in place (pair c into x[c]) and
+      // summed as rounded; with want_max, the row's max is taken from the same reads
+      auto exp_pass = [&](float m_used, bool want_max) {
+        const float nms = -m_used * eff;
+        const uint64_t nms2 = tg::f2_pack(nms, nms);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(x[k]);
+        for (int k = 0; k < 8; ++k) {
+          acc[k] = 0.f;
+          mx[k] = -INFINITY;
+        }
 #pragma unroll
-      for (int c = 8; c < kBN; c += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = tg::fmax3(mx[k], __uint_as_float(x[c + k]), __uint_as_float(x[c + 8 + k]));
-      const float rmax = fmaxf(tg::fmax3(mx[0], mx[1], mx[2]), tg::fmax3(tg::fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
-      const float m_new = fmaxf(m, rmax);
-      // taken per warp: the TMEM loads and stores of the rescale are warp-collective
-      const bool rescale = __any_sync(0xFFFFFFFFu, (m_new - m) * eff > kRescaleLog2);
+        for (int c = 0; c < kBN / 2; ++c) {
+          const float s0 = __uint_as_float(x[2 * c]), s1 = __uint_as_float(x[2 * c + 1]);
+          if (want_max) mx[c & 7] = tg::fmax3(mx[c & 7], s0, s1);
+          const uint64_t arg = tg::f2_fma(tg::f2_pack(s0, s1), eff2, nms2);
+          float a0, a1;
+          tg::f2_unpack(arg, a0, a1);
+          const uint32_t pb = pack_bf16x2(tg::ex2_approx(a0), tg::ex2_approx(a1));
+          x[c] = pb;  // in place: x[c] is no longer needed once read above
+          // the row sum adds the same bf16-rounded weights the PV product uses, so every
+          // output row is an exact convex combination of its value rows
+          tg::add_bf16x2_to_f32(acc[(2 * c) & 7], acc[(2 * c + 1) & 7], pb);
+        }
+      };
+      auto row_max = [&]() {
+        return fmaxf(tg::fmax3(mx[0], mx[1], mx[2]), tg::fmax3(tg::fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+      };
+      load_row();
       float alpha = 1.f;
-      if (rescale) {
-        alpha = tg::ex2_approx((m - m_new) * eff);
-        m = m_new;
-      }
-      const float nms = -m * eff;
-      const uint64_t nms2 = tg::f2_pack(nms, nms);
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      bool rescale;
+      if (j == 0) {
+        // first tile: the max first (there is no running max to use yet); 8 running maxima
+        // over the 64 pairs of the row
 #pragma unroll
-      for (int c = 0; c < kBN / 2; ++c) {
-        const uint64_t arg = tg::f2_fma(tg::f2_pack(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), eff2, nms2);
-        float a0, a1;
-        tg::f2_unpack(arg, a0, a1);
-        const uint32_t pb = pack_bf16x2(tg::ex2_approx(a0), tg::ex2_approx(a1));
-        x[c] = pb;  // in place: x[c] is no longer needed once read above
-        // the row sum adds the same bf16-rounded weights the PV product uses, so every
-        // output row is an exact convex combination of its value rows
-        tg::add_bf16x2_to_f32(acc[(2 * c) & 7], acc[(2 * c + 1) & 7], pb);
+        for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBN / 2; ++c)
+          mx[c & 7] = tg::fmax3(mx[c & 7], __uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1]));
+        const float m_new = fmaxf(m, row_max());
+        // taken per warp: the TMEM loads and stores of the rescale are warp-collective
+        rescale = __any_sync(0xFFFFFFFFu, (m_new - m) * eff > kRescaleLog2);
+        if (rescale) {
+          alpha = tg::ex2_approx((m - m_new) * eff);
+          m = m_new;
+        }
+        exp_pass(m, false);
+      } else {
+        // exponentials against the running max, the tile's max taken in the same pass (the
+        // max then costs no time of its own: the pass waits on the MUFU); only when the max
+        // grows past the rescale threshold is the row read again from TMEM and redone
+        exp_pass(m, true);
+        const float m_new = fmaxf(m, row_max());
+        rescale = __any_sync(0xFFFFFFFFu, (m_new - m) * eff > kRescaleLog2);
+        if (rescale) {
+          alpha = tg::ex2_approx((m - m_new) * eff);
+          m = m_new;
+          load_row();
+          exp_pass(m, false);
+        }
       }
       tg::tmem_st32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
       tg::tmem_st32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));

@@ -88,8 +88,9 @@ inline Workspace carve(void *base, int64_t S, int32_t Hq) {
 }
 
 // ------------------------------------------------------------------------------ prep
-// One warp per (row, head) of the padded range: Delta = dO . O (fp32), and
-// the lse converted to base 2; both stored negated, per head.
+// One warp per (row, head) of the padded range, the whole range in one grid: Delta =
+// dO . O (fp32), from the fp32 output with one 16-byte load per lane (D = 128) when it
+// is given, and the lse converted to base 2; both stored negated, per head.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16 *__restrict__ O,
                                                             const float *__restrict__ O32,
@@ -98,45 +99,60 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16 
                                                             int Hq, Workspace ws) {
   tg::pdl_wait();
   tg::pdl_trigger();
+  constexpr int kPer = D / 32;  // elements per lane (2 or 4)
   const int lane = threadIdx.x & 31;
-  const int64_t n_rows = S_pad * Hq;
-  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < n_rows;
-       w += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
-    const int64_t i = w / Hq;
-    const int h = static_cast<int>(w % Hq);
-    float nd = 0.f, nl = -INFINITY;
-    if (i < S) {
-      constexpr int kPer = D / 32;  // bf16 elements per lane (2 or 4)
-      const __nv_bfloat16 *d = dO + (i * Hq + h) * D + lane * kPer;
-      float acc = 0.f;
-      if (O32) {
-        const float *o32 = O32 + (i * Hq + h) * D + lane * kPer;
-#pragma unroll
-        for (int e = 0; e < kPer; e += 2) {
-          const float2 a = *reinterpret_cast<const float2 *>(o32 + e);
-          const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(d + e);
-          acc = fmaf(a.x, __low2float(b), acc);
-          acc = fmaf(a.y, __high2float(b), acc);
-        }
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (w >= S_pad * Hq) return;  // whole warps
+  const int64_t i = w / Hq;
+  const int h = static_cast<int>(w % Hq);
+  float nd = 0.f, nl = -INFINITY;
+  if (i < S) {
+    const int64_t off = (i * Hq + h) * D + lane * kPer;
+    float o[kPer], d[kPer];
+    if constexpr (kPer == 4) {
+      const uint2 dv = *reinterpret_cast<const uint2 *>(dO + off);
+      const __nv_bfloat162 d01 = *reinterpret_cast<const __nv_bfloat162 *>(&dv.x);
+      const __nv_bfloat162 d23 = *reinterpret_cast<const __nv_bfloat162 *>(&dv.y);
+      d[0] = __low2float(d01);
+      d[1] = __high2float(d01);
+      d[2] = __low2float(d23);
+      d[3] = __high2float(d23);
+    } else {
+      const __nv_bfloat162 d01 = *reinterpret_cast<const __nv_bfloat162 *>(dO + off);
+      d[0] = __low2float(d01);
+      d[1] = __high2float(d01);
+    }
+    if (O32) {
+      if constexpr (kPer == 4) {
+        const float4 ov = *reinterpret_cast<const float4 *>(O32 + off);
+        o[0] = ov.x;
+        o[1] = ov.y;
+        o[2] = ov.z;
+        o[3] = ov.w;
       } else {
-        const __nv_bfloat16 *o = O + (i * Hq + h) * D + lane * kPer;
-#pragma unroll
-        for (int e = 0; e < kPer; e += 2) {
-          const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(o + e);
-          const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(d + e);
-          acc = fmaf(__low2float(a), __low2float(b), acc);
-          acc = fmaf(__high2float(a), __high2float(b), acc);
-        }
+        const float2 ov = *reinterpret_cast<const float2 *>(O32 + off);
+        o[0] = ov.x;
+        o[1] = ov.y;
       }
+    } else {
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-      nd = -acc;
-      nl = -lse[i * Hq + h] * kLog2e;
+      for (int e = 0; e < kPer; e += 2) {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(O + off + e);
+        o[e] = __low2float(a);
+        o[e + 1] = __high2float(a);
+      }
     }
-    if (lane == 0) {
-      ws.ndelta[h * S_pad + i] = nd;
-      ws.nlse2[h * S_pad + i] = nl;
-    }
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc = fmaf(o[e], d[e], acc);
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, sh);
+    nd = -acc;
+    nl = -lse[i * Hq + h] * kLog2e;
+  }
+  if (lane == 0) {
+    ws.ndelta[h * S_pad + i] = nd;
+    ws.nlse2[h * S_pad + i] = nl;
   }
 }
 
@@ -424,8 +440,8 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
                       "needs 168", fa.numRegs);
     configured[dev] = true;
   }
-  const int64_t prep_warps = S_pad * Hq;
-  const unsigned prep_grid = static_cast<unsigned>(std::min<int64_t>((prep_warps + 7) / 8, 8LL * tg::sm_count()));
+  const int64_t prep_warps = S_pad * Hq;  // below 2^31 (checked by the caller)
+  const unsigned prep_grid = static_cast<unsigned>((prep_warps + 7) / 8);
   cudaError_t e = tg::launch_pdl(attn_bwd_prep_kernel<D>, dim3(prep_grid), dim3(256), 0, stream,
                                  reinterpret_cast<const __nv_bfloat16 *>(O), O32,
                                  reinterpret_cast<const __nv_bfloat16 *>(dO), lse, S, S_pad, static_cast<int>(Hq), ws);

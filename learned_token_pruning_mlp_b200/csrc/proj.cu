@@ -15,8 +15,8 @@
 // consecutive tiles sharing the same 256 rows of x.  The elementwise work sits in the
 // epilogue, run by two warpgroups per CTA (each thread owns one row, i.e. one TMEM
 // lane, and half of the tile's columns):
-//   * output projection: + residual, whose rows are prefetched into L2 before the
-//     accumulator is ready;
+//   * output projection: + residual, whose row slice each thread loads into registers
+//     before the accumulator is ready;
 //   * QKV: a 256-column tile holds whole heads of one kind (Q, K or V).  The tile is
 //     four (head, 32-pair chunk) units; each warpgroup takes the two units that share
 //     one chunk of rotary indices j, so each thread forms 32 angles per tile and
@@ -216,12 +216,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int64_t row = mt * 2 * kBM + rank * kBM + quarter * 32 + lane;
       const bool row_ok = row < M;
       const int n0 = nt * kBN;
+      // the residual slice this thread adds (its row, the group's 128 columns), loaded into
+      // registers before the accumulator is ready so the loads overlap the tile's MMAs
+      uint4 res[kHD == 0 ? 16 : 1];
       if constexpr (kHD == 0) {
-        // the residual slice this thread adds, pulled into L2 while the MMA runs
         const int c0 = n0 + group * (kBN / 2);
-        if (out.residual && row_ok && c0 < N)
-          tg::prefetch_l2(out.residual + row * static_cast<int64_t>(N) + c0,
-                          static_cast<uint32_t>(min(kBN / 2, N - c0)) * 2u);
+        if (out.residual && row_ok) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(out.residual + row * static_cast<int64_t>(N) + c0);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) res[q] = c0 + 8 * q < N ? src[q] : make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       int32_t p = 0;
       if constexpr (kHD > 0) p = row_ok ? out.pos[row] : 0;
@@ -229,7 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tg::tc_fence_after();
       const uint32_t taddr = tmem_base + acc * static_cast<uint32_t>(kBN) + (static_cast<uint32_t>(quarter * 32) << 16);
       if constexpr (kHD == 0) {
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < kBN / 64; ++c) {
           const int cc = group * (kBN / 64) + c;  // 32-column chunk of the tile
           uint32_t r[32];
@@ -241,13 +245,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (out.residual) {
-              const uint4 *src = reinterpret_cast<const uint4 *>(out.residual + row * static_cast<int64_t>(N) + col);
-              uint4 u[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) u[q] = src[q];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+                const uint4 u = res[4 * c + q];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
