@@ -251,6 +251,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = tg::idesc_bf16_f32(kBK, kBQ, false, false);
+    // shared-memory descriptors built once; each K step adds its constant offset to the
+    // start-address field of the low word (16-byte units; shared addresses stay below
+    // 2^18 bytes, so the add never carries out of the 14-bit field)
+    const uint64_t dk = tg::smem_desc_sw128(tg::smem_addr(sK), 16, 1024);
+    const uint32_t hi = static_cast<uint32_t>(dk >> 32), k_lo = static_cast<uint32_t>(dk);
+    const uint32_t v_lo = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sV), 16, 1024));
+    const uint32_t q_lo0 = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sQ), 16, 1024));
+    const uint32_t do_lo0 = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sdO), 16, 1024));
+    constexpr uint32_t kTileUnits = C::kTileBytes >> 4;
     bool ok = tg::mbar_wait(tg::smem_addr(&ctl->kv_full), 0, abort_flag);
     for (int n = 0; n < n_steps && ok; ++n) {
       const int s = n % NS;
@@ -259,18 +268,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->tmem_empty[buf]), ((n >> 1) & 1) ^ 1, abort_flag))) break;
       tg::tc_fence_after();
       const uint32_t d_s = tmem_base + static_cast<uint32_t>(buf * 256);
+      const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(s) * kTileUnits;
+      const uint32_t do_lo = do_lo0 + static_cast<uint32_t>(s) * kTileUnits;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
-        tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(tg::smem_addr(sK) + off, 16, 1024),
-                        tg::smem_desc_sw128(tg::smem_addr(sQ + s * C::kTileBytes) + off, 16, 1024), idesc,
-                        kk > 0 ? 1u : 0u);
+        const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+        tg::mma_bf16_ss(d_s, tg::desc_words(k_lo + off, hi), tg::desc_words(q_lo + off, hi), idesc, kk > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = static_cast<uint32_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32);
-        tg::mma_bf16_ss(d_s + kBQ, tg::smem_desc_sw128(tg::smem_addr(sV) + off, 16, 1024),
-                        tg::smem_desc_sw128(tg::smem_addr(sdO + s * C::kTileBytes) + off, 16, 1024), idesc,
+        const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+        tg::mma_bf16_ss(d_s + kBQ, tg::desc_words(v_lo + off, hi), tg::desc_words(do_lo + off, hi), idesc,
                         kk > 0 ? 1u : 0u);
       }
       tg::mma_commit(tg::smem_addr(&ctl->s_full[buf]));
