@@ -407,20 +407,46 @@ def run_e2e(tg, host, dev, w, K, S, tau, world, args):
         sum(t.numel() * t.element_size() for lay in h_layers for t in lay)
     d2h = h_kept.numel() * 4 + sum(o.numel() * o.element_size() for o in h_outs)
 
+    comp = torch.cuda.current_stream(dev)
+    h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
     def step():
-        for k in h_in:
-            d_in[k].copy_(h_in[k], non_blocking=True)
-        for l in range(L):
-            for a, b in zip(d_layers[l], h_layers[l]):
-                a.copy_(b, non_blocking=True)
+        # Host-to-device copies on their own stream (the select path's inputs, then each
+        # layer's Q/K/V in order), device-to-host reads of each result on another, so the
+        # copies overlap the kernels; a step starts after the previous one has finished
+        # (its device buffers are reused) and ends when its results are on the host.
+        h2d_stream.wait_stream(comp)
+        layer_ready = []
+        with torch.cuda.stream(h2d_stream):
+            for k in h_in:
+                d_in[k].copy_(h_in[k], non_blocking=True)
+            inputs_ready = torch.cuda.Event()
+            inputs_ready.record(h2d_stream)
+            for l in range(L):
+                for a, b in zip(d_layers[l], h_layers[l]):
+                    a.copy_(b, non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(h2d_stream)
+                layer_ready.append(e)
+        comp.wait_event(inputs_ready)
         tg.tg_gate_score(d_in["hidden"], d_in["W1"], d_in["b1"], d_in["W2"], d_in["b2"], scores=scores)
         tg.tg_select_topk(d_in["sel"], d_in["mask"], K, kept_idx=kept, n_kept=n_kept)
         tg.tg_gather(d_in["hidden"], kept, n_rows=S, n_kept=n_kept, hidden_k=hidden_k, scores=d_in["sel"], s_k=s_k)
+        sel_done = torch.cuda.Event()
+        sel_done.record(comp)
+        d2h_stream.wait_event(sel_done)
+        with torch.cuda.stream(d2h_stream):
+            h_kept.copy_(kept[:S], non_blocking=True)
         for l in range(L):
+            comp.wait_event(layer_ready[l])
             Q, Kc, V = d_layers[l]
             tg.tg_gated_attention(Q, Kc, V, s_k, d_in["gain"], tau, O=outs[l])
-            h_outs[l].copy_(outs[l], non_blocking=True)
-        h_kept.copy_(kept[:S], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(comp)
+            d2h_stream.wait_event(done)
+            with torch.cuda.stream(d2h_stream):
+                h_outs[l].copy_(outs[l], non_blocking=True)
+        comp.wait_stream(d2h_stream)
 
     steps = max(1, min(args.steps, 3))
     step()
@@ -428,10 +454,10 @@ def run_e2e(tg, host, dev, w, K, S, tau, world, args):
     barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
+    t0.record(comp)
     for _ in range(steps):
         step()
-    t1.record()
+    t1.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
     flops = attention_flops(S, w.hq, w.head_dim) * L
