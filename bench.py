@@ -10,6 +10,8 @@ whole step (27 layers of 4*D*Hq*S*(S+1)/2 flops divided by the full step time, t
 gate/top-K/gather time included); the gate+top-K+gather path is reported beside
 it in GB/s against HBM.  Inputs are resident in HBM before timing starts; the
 per-step working set (512 MiB residual + 1.9 GB of Q/K/V) is larger than L2.
+``attention.context`` compares, outside the timed step, the kernel with and without
+the key bias and the library's causal attention on the same layers.
 ``next_rows`` gives the device time of the calls around the path on the same
 workload, outside the timed step: the pruned layer's projections, the attention
 backward, random-K and a 4-budget sweep.
@@ -292,6 +294,7 @@ def run_tokengate(args, world, rank, local):
     # from pinned memory and D2H of its results inside the timed region
     e2e = run_e2e(tg, host, dev, w, K, S, tau, world, args)
     next_rows = time_next_rows(tg, dev, w, host, dv, kept, S)
+    attn_ctx = attention_context(tg, dev, w, layers, s_k, dv["gain"], tau, S)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -301,7 +304,7 @@ def run_tokengate(args, world, rank, local):
         "attention": {"ms_per_layer": round(att_launch_ms, 4), "tflops": round(att_tflops, 1),
                       "frac_of_bf16_peak": round(att_tflops / peaks["bf16_tflops"], 4),
                       "frac_of_bf16_sustained": round(att_tflops / peaks["bf16_tflops_sustained"], 4),
-                      "frac_of_nominal_2250": round(att_tflops / 2250.0, 4)},
+                      "frac_of_nominal_2250": round(att_tflops / 2250.0, 4), "context": attn_ctx},
         "select_path": {"us": round(sel_b2b_us, 2), "bytes": sel_bytes, "gbs": round(sel_b2b_gbs, 1),
                         "frac_of_hbm": round(sel_b2b_gbs / peaks["hbm_gbs"], 4),
                         "frac_of_datasheet_8tbs": round(sel_b2b_gbs / DATASHEET_HBM_GBS, 4),
@@ -320,6 +323,52 @@ def run_tokengate(args, world, rank, local):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(host, w, S, budget_s=args.cpu_seconds)
+    return out
+
+
+def attention_context(tg, dev, w, layers, s_k, gain, tau, S):
+    """Per-layer time of the attention over the step's 27 layers (inputs larger than L2):
+    the gated kernel, the same kernel without the key bias (plain causal attention), and,
+    as context only, the library's causal attention (torch scaled_dot_product_attention)
+    without and with an additive bias mask.  Outside the timed step."""
+    stream = torch.cuda.current_stream(dev)
+    L = len(layers)
+    outs = [torch.empty(S, w.hq, w.head_dim, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+
+    def per_layer_us(fn, n_layers):
+        for i in range(min(3, n_layers)):
+            fn(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_layers):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n_layers * 1e3
+
+    gated = per_layer_us(lambda i: tg.tg_gated_attention(*layers[i], s_k, gain, tau, O=outs[i & 1]), L)
+    plain = per_layer_us(lambda i: tg.tg_gated_attention(*layers[i], None, None, tau, O=outs[i & 1]), L)
+    out = {"gated_us_per_layer": round(gated, 2), "no_bias_us_per_layer": round(plain, 2),
+           "bias_overhead": round(gated / plain, 4)}
+    try:
+        import torch.nn.functional as F
+        n_lib = min(L, 6)
+        lib_layers = [tuple(t.transpose(0, 1).unsqueeze(0).contiguous() for t in layers[i]) for i in range(n_lib)]
+        scale = tau / math.sqrt(w.head_dim)
+        sdpa = per_layer_us(lambda i: F.scaled_dot_product_attention(
+            *lib_layers[i % n_lib], is_causal=True, scale=scale, enable_gqa=True), n_lib * 2)
+        # an additive mask: causal -inf plus the bias of head 0 on every head (one mask)
+        bias = (gain[0] * s_k).to(torch.bfloat16)
+        mask = torch.full((S, S), float("-inf"), device=dev, dtype=torch.bfloat16).triu(1) + bias[None, :]
+        sdpa_b = per_layer_us(lambda i: F.scaled_dot_product_attention(
+            *lib_layers[i % n_lib], attn_mask=mask[None, None], scale=scale, enable_gqa=True), n_lib * 2)
+        out.update({"library_sdpa_causal_us_per_layer": round(sdpa, 2),
+                    "library_sdpa_bias_mask_us_per_layer": round(sdpa_b, 2),
+                    "library": f"torch {torch.__version__} scaled_dot_product_attention, bf16, GQA"})
+        del lib_layers, mask
+    except Exception as exc:  # context only: report why it is missing
+        out["library"] = f"unavailable: {type(exc).__name__}: {exc}"[:200]
     return out
 
 

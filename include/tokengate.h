@@ -225,7 +225,10 @@ tg_status tg_gather(const tg_bf16 *hidden, int64_t n, int32_t d, const int32_t *
  * indices are ascending.  bf16 inputs, fp32 accumulation, bf16 output.
  *
  *   Q   bf16 [S, Hq, D]    Kc, V  bf16 [S, Hkv, D]    O  bf16 [S, Hq, D]
- *   s   fp32 [S]           gain   fp32 [Hq]           tau (host float)
+ *   s   fp32 [S] or NULL   gain   fp32 [Hq]           tau (host float)
+ * With s = NULL the call is plain causal GQA attention (no key bias; gain may then
+ * also be NULL): the form of the layers below the gate, and the baseline the bias
+ * costs are measured against.
  * Sizes: S >= 0; D in {64, 128}; Hq a positive multiple of Hkv; S * Hq < 2^31.
  * Q, Kc, V and O 16-byte aligned.
  * -------------------------------------------------------------------------- */

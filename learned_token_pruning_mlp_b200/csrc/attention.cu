@@ -7,6 +7,8 @@
 // head h, KV head g = h / (Hq/Hkv):
 //     logit(i,j) = tau * Q[i,h].K[j,g] / sqrt(D) + gain[h] * s[j]   (j <= i)
 //     O[i,h]     = softmax_j(logit(i,.)) V[., g]
+// Without scores (s = NULL) the call is plain causal GQA attention: the kernel
+// instantiation without the bias step runs (tau = 0 keeps it, with a block of zeros).
 //
 // B200 design (flash-style, one CTA per pair of 128-row query tiles of one head):
 //   * TMEM (512 columns): S_0, S_1 (128 fp32 columns each, one per query tile),
@@ -91,7 +93,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int D>
+// kBias: the key-bias step is part of every S' product (with scores, or with tau = 0
+// where it is the whole product); without it the kernel is plain causal attention.
+template <int D, bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     gated_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ key_scores,
@@ -136,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- logit scaling: base-2 logit = eff * S', S' = (+/-)(q.k + c_j)
   const bool skip_qk = (scale_log2 == 0.f);
   const float eff = skip_qk ? 1.f : fabsf(scale_log2);
-  const float cmul = gain[h] * kLog2e / (skip_qk ? 1.f : scale_log2);
+  const bool has_bias = key_scores != nullptr;  // kBias without scores: a block of zeros
+  const float cmul = has_bias ? gain[h] * kLog2e / (skip_qk ? 1.f : scale_log2) : 0.f;
 
   const int warp = tg::warp_id();
   const int lane = threadIdx.x & 31;
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < kBN / 32; ++e) {
         const int r = e * 32 + lane;
         const int64_t kv = static_cast<int64_t>(j) * kBN + r;
-        const float c = kv < len ? cmul * key_scores[seg_start + kv] : 0.f;
+        const float c = has_bias && kv < len ? cmul * key_scores[seg_start + kv] : 0.f;
         const __nv_bfloat16 hi = __float2bfloat16_rn(c);
         const __nv_bfloat16 lo = __float2bfloat16_rn(c - __bfloat162float(hi));
         const __nv_bfloat162 pr = __halves2bfloat162(hi, lo);
@@ -254,13 +259,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_s = [&](int t, int j) {
       const uint32_t s = static_cast<uint32_t>(j % NS);
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(t * kBN);
-      tg::mma_bf16_ss(d_tmem, dqx, tg::desc_words(kx_lo0 + s * (kExtBytes >> 4), hi_x), idesc_s, 0u);
+      if constexpr (kBias) tg::mma_bf16_ss(d_tmem, dqx, tg::desc_words(kx_lo0 + s * (kExtBytes >> 4), hi_x), idesc_s, 0u);
       if (!skip_qk) {
         const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(t) * kTileUnits, k_lo = k_lo0 + s * kTileUnits;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
-          tg::mma_bf16_ss(d_tmem, tg::desc_words(q_lo + off, hi_sw), tg::desc_words(k_lo + off, hi_sw), idesc_s, 1u);
+          tg::mma_bf16_ss(d_tmem, tg::desc_words(q_lo + off, hi_sw), tg::desc_words(k_lo + off, hi_sw), idesc_s,
+                          (kBias || kk > 0) ? 1u : 0u);
         }
       }
       tg::mma_commit(tg::smem_addr(&ctl->s_full[t]));
@@ -474,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
-tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain, float tau,
+template <int D, bool kBias>
+tg_status launch_kernel(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain, float tau,
                  const int32_t *cu_seqlens, int32_t B, int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv,
                  tg_bf16 *O, float *lse, float *O32, cudaStream_t stream, uint32_t *err) {
   using C = Cfg<D>;
@@ -500,12 +506,12 @@ tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const fl
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(gated_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(gated_attention_kernel<D, kBias>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     // the warpgroup register split in the kernel assumes 168 registers per thread at launch
     cudaFuncAttributes fa;
-    const cudaError_t ea = cudaFuncGetAttributes(&fa, gated_attention_kernel<D>);
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, gated_attention_kernel<D, kBias>);
     if (ea != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(ea));
     if (fa.numRegs != 168)
       return tg::fail(TG_ERR_UNSUPPORTED, "gated_attention_kernel built with %d registers per thread; the register "
@@ -517,12 +523,24 @@ tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const fl
   const int64_t grid = static_cast<int64_t>(n_mblocks) * Hq * B;
   if (grid == 0) return TG_OK;
   if (grid > 0x7FFFFFFFLL) return tg::fail(TG_ERR_UNSUPPORTED, "grid too large");
-  const cudaError_t e = tg::launch_pdl(gated_attention_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+  const cudaError_t e = tg::launch_pdl(gated_attention_kernel<D, kBias>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
                                       C::kSmem, stream, tm_q, tm_k, tm_v, s, gain, scale_log2, cu_seqlens,
                                       cu_seqlens ? int64_t(0) : total, total, n_mblocks, B, Hq, Hkv,
                                       reinterpret_cast<__nv_bfloat16 *>(O), lse, O32, err);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gated_attention_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("gated_attention_kernel");
+}
+
+template <int D>
+tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain, float tau,
+                 const int32_t *cu_seqlens, int32_t B, int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv,
+                 tg_bf16 *O, float *lse, float *O32, cudaStream_t stream, uint32_t *err) {
+  // plain causal attention leaves the bias step out; with tau = 0 it is the whole product
+  if (s || tau == 0.f)
+    return launch_kernel<D, true>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, lse, O32,
+                                  stream, err);
+  return launch_kernel<D, false>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, lse, O32,
+                                 stream, err);
 }
 
 tg_status validate(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain,
@@ -534,7 +552,8 @@ tg_status validate(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const 
   if (!std::isfinite(tau)) return tg::fail(TG_ERR_INVALID_ARG, "tau must be finite");
   if (total * Hq >= 0x7FFFFFFFLL) return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
   if (total == 0) return TG_OK;
-  if (!Q || !Kc || !V || !s || !gain || !O) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (!Q || !Kc || !V || !O) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (s && !gain) return tg::fail(TG_ERR_INVALID_ARG, "gain is NULL");
   if (!tg::aligned16(Q) || !tg::aligned16(Kc) || !tg::aligned16(V) || !tg::aligned16(O))
     return tg::fail(TG_ERR_ALIGNMENT, "Q, Kc, V and O must be 16-byte aligned");
   return TG_OK;

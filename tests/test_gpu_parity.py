@@ -378,3 +378,18 @@ def test_bounded_wait_times_out_and_context_survives():
     x = torch.randn(1000, device=DEV)
     assert torch.isfinite(x.sum()).item()
     test_gather_bit_exact(37, 8, 37)
+
+
+# =============================================================================== no key bias
+@pytest.mark.parametrize("S,Hq,Hkv,D,tau", [(700, 16, 8, 128, 1.1), (300, 4, 2, 64, 2.5), (129, 2, 1, 128, -0.7),
+                                            (200, 4, 2, 64, 0.0)])
+def test_attention_without_scores_is_plain_causal_attention(S, Hq, Hkv, D, tau):
+    """s = NULL: the oracle's definition with a zero bias (tau = 0: uniform weights)."""
+    g = torch.Generator().manual_seed(S + D)
+    Q = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    K = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    O = tg.tg_gated_attention(Q.to(DEV), K.to(DEV), V.to(DEV), None, None, tau)
+    ref = oracle.gated_attention(Q, K, V, np.zeros(S, np.float32), np.zeros(Hq, np.float32), tau)
+    assert_attn_close(O.float().cpu().numpy(), ref)
+    assert _devbits() == 0
