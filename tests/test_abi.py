@@ -100,7 +100,7 @@ def test_attention_rejects_bad_arguments(L):
     assert L.tg_gated_attention(p, p, p, p, p, f, 10, 4, 2, 96, p, None) == 2              # D
     assert L.tg_gated_attention(p, p, p, p, p, ctypes.c_float(float("inf")), 10, 4, 2, 64, p, None) == 1
     assert L.tg_gated_attention(p, p, p, p, p, f, 0, 4, 2, 64, p, None) == 0               # S = 0
-    assert L.tg_gated_attention(p, p, p, None, p, f, 10, 4, 2, 64, p, None) == 1
+    assert L.tg_gated_attention(p, p, p, p, None, f, 10, 4, 2, 64, p, None) == 1            # scores without gain
     assert L.tg_gated_attention(ctypes.c_void_p(4104), p, p, p, p, f, 10, 4, 2, 64, p, None) == 3
     assert L.tg_gated_attention_varlen(p, p, p, p, p, f, None, 2, 10, 5, 4, 2, 64, p, None) == 1
     assert L.tg_gated_attention_varlen(p, p, p, p, p, f, p, 2, 10, 11, 4, 2, 64, p, None) == 1
