@@ -22,7 +22,12 @@
 //     a bias.  tau < 0 negates the A operand (so the largest logit is still the
 //     largest S'); tau = 0 skips the Q.K steps.
 //   * warp 0 (one lane) loads Q once and streams K/V tiles of 128 keys through a
-//     TMA pipeline (128-byte swizzle); warp 3 writes the c_j block of each tile into
+//     TMA pipeline (128-byte swizzle).  K and V stages are freed apart: a K stage as
+//     soon as the S' products of its tile complete, a V stage when its PV products do,
+//     so each K load has a whole KV step to land before its product is issued (with
+//     one release per K/V pair, the next K load could only start once the tile after
+//     it had been multiplied, and the tensor core waited on it every step); warp 3
+//     writes the c_j block of each tile into
 //     shared memory from plain loads of the scores (request offsets need not be
 //     16-byte aligned, which a TMA copy would require).
 //   * warp 1 (one lane) issues every tcgen05.mma: S_t = [1 Q] [c K]^T (K-major
@@ -78,7 +83,8 @@ struct AttnCtl {
   uint64_t q_full;
   uint64_t k_full[4];
   uint64_t v_full[4];
-  uint64_t kv_empty[4];
+  uint64_t k_empty[4];
+  uint64_t v_empty[4];
   uint64_t bias_full[4];
   uint64_t s_full[2];
   uint64_t p_full[2];
@@ -98,7 +104,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int D, bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     gated_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ key_scores,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                           const float *__restrict__ key_scores,
                            const float *__restrict__ gain, float scale_log2, const int32_t *__restrict__ cu_seqlens,
                            int64_t S_single, int64_t total, int n_mblocks, int B, int Hq, int Hkv,
                            __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, float *__restrict__ O32,
@@ -159,7 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < NS; ++s) {
       tg::mbar_init(tg::smem_addr(&ctl->k_full[s]), 1);
       tg::mbar_init(tg::smem_addr(&ctl->v_full[s]), 1);
-      tg::mbar_init(tg::smem_addr(&ctl->kv_empty[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->k_empty[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->v_empty[s]), 1);
       tg::mbar_init(tg::smem_addr(&ctl->bias_full[s]), 32);
     }
     for (int t = 0; t < 2; ++t) {
@@ -173,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::prefetch_tmap(&tm_q);
     tg::prefetch_tmap(&tm_k);
     tg::prefetch_tmap(&tm_v);
+    tg::prefetch_tmap(&tm_o);
   }
   if (warp == 2) {
     tg::tmem_alloc(tg::smem_addr(&ctl->tmem_base), 512);
@@ -203,12 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n_kv; ++j) {
       const int s = j % NS;
       const uint32_t ph = (j / NS) & 1;
-      if (!tg::mbar_wait(tg::smem_addr(&ctl->kv_empty[s]), ph ^ 1u, abort_flag)) break;
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->k_empty[s]), ph ^ 1u, abort_flag)) break;
       const int32_t krow = static_cast<int32_t>(seg_start + static_cast<int64_t>(j) * kBN);
       const uint32_t kb = tg::smem_addr(&ctl->k_full[s]);
       tg::mbar_arrive_expect_tx(kb, C::kTileBytes);
       for (int hf = 0; hf < C::kHalves; ++hf)
         tg::tma_load_3d(tg::smem_addr(sK + s * C::kTileBytes + hf * kHalfBytes), &tm_k, kb, hf * 64, g, krow);
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->v_empty[s]), ph ^ 1u, abort_flag)) break;
       const uint32_t vb = tg::smem_addr(&ctl->v_full[s]);
       tg::mbar_arrive_expect_tx(vb, C::kTileBytes);
       for (int hf = 0; hf < C::kHalves; ++hf)
@@ -219,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n_kv; ++j) {
       const int s = j % NS;
       const uint32_t ph = (j / NS) & 1;
-      if (!tg::mbar_wait(tg::smem_addr(&ctl->kv_empty[s]), ph ^ 1u, abort_flag)) break;
+      if (!tg::mbar_wait(tg::smem_addr(&ctl->k_empty[s]), ph ^ 1u, abort_flag)) break;
 #pragma unroll
       for (int e = 0; e < kBN / 32; ++e) {
         const int r = e * 32 + lane;
@@ -292,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::tc_fence_after();
       issue_s(0, 0);
       if (n1) issue_s(1, 0);
+      tg::mma_commit(tg::smem_addr(&ctl->k_empty[0]));
     }
     for (int j = 0; j < n_kv && ok; ++j) {
       const int s = j % NS;
@@ -312,13 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->p_full[1]), j & 1u, abort_flag))) break;
         tg::tc_fence_after();
         issue_pv(1, j);
-        if (j + 1 < n1) {
-          if (!next_k_ready && !(ok = wait_k(j + 1))) break;
-          tg::tc_fence_after();
-          issue_s(1, j + 1);
-        }
       }
-      tg::mma_commit(tg::smem_addr(&ctl->kv_empty[s]));
+      tg::mma_commit(tg::smem_addr(&ctl->v_empty[s]));  // V_j's last product
+      if (j + 1 < n1) {
+        if (!next_k_ready && !(ok = wait_k(j + 1))) break;
+        tg::tc_fence_after();
+        issue_s(1, j + 1);
+      }
+      if (j + 1 < n_kv) tg::mma_commit(tg::smem_addr(&ctl->k_empty[(j + 1) % NS]));  // K_{j+1}'s last product
     }
     if (ok) tg::mma_commit(tg::smem_addr(&ctl->o_final));
     if (*abort_flag) {
@@ -439,6 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::tc_fence_before();
       tg::mbar_arrive(tg::smem_addr(&ctl->p_full[t]));
     }
+    // A whole tile of bf16 output leaves through shared memory and a tensor store:
+    // the rows are staged in the 128-byte-swizzled layout the tensor map expects, over
+    // this tile's Q buffer (every product has completed), and written as full 128-byte
+    // lines.  A partial tile (its rows past the end of the request may belong to the
+    // next one) and the fp32 copy are stored row by row.
+    const bool staged = !O32 && rt + kBM <= len;  // uniform over the warpgroup
+    uint8_t *stage = sQ + t * C::kTileBytes;
     if (ok && n_t > 0 && tg::mbar_wait_warp(tg::smem_addr(&ctl->o_final), 0, abort_flag)) {
       tg::tc_fence_after();
       const float inv_l = 1.0f / l;
@@ -455,6 +474,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (staged) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = (c & 1) * 4 + q;  // 16-byte chunk within the 64-column half c / 2
+            *reinterpret_cast<uint4 *>(stage + (c >> 1) * kHalfBytes + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+          continue;
+        }
         if (O32 && row < len) {
           float4 *d32 = reinterpret_cast<float4 *>(O32 + ((seg_start + row) * Hq + h) * static_cast<int64_t>(D) + c * 32);
 #pragma unroll
@@ -467,6 +495,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
+      }
+    }
+    if (staged) {
+      // every warp of the warpgroup arrives here, also after a failed wait (no store then)
+      tg::fence_proxy_async_smem();
+      if (t == 0) asm volatile("bar.sync 1, 128;" ::: "memory");  // this warpgroup's rows are staged
+      else asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (quarter == 0 && lane == 0 && !*abort_flag) {
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tg::tma_store_3d(&tm_o, tg::smem_addr(stage + hf * kHalfBytes), hf * 64, h,
+                           static_cast<int32_t>(seg_start + rt));
+        tg::bulk_commit();
+        tg::bulk_wait_read_all();  // the staging buffer is read before the CTA exits
       }
     }
   }
@@ -485,12 +526,15 @@ tg_status launch_kernel(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, c
                  const int32_t *cu_seqlens, int32_t B, int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv,
                  tg_bf16 *O, float *lse, float *O32, cudaStream_t stream, uint32_t *err) {
   using C = Cfg<D>;
-  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_q, tm_k, tm_v, tm_o;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(Hq), static_cast<uint64_t>(total)};
     const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hq) * D * 2};
     const uint32_t box[3] = {64, 1, kBM};
     if (!tg::encode_tmap(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return TG_ERR_CUDA;
+    // O has Q's shape; its map serves the tensor stores of whole output tiles
+    if (!tg::encode_tmap(&tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, O, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return TG_ERR_CUDA;
   }
   {
@@ -524,7 +568,7 @@ tg_status launch_kernel(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, c
   if (grid == 0) return TG_OK;
   if (grid > 0x7FFFFFFFLL) return tg::fail(TG_ERR_UNSUPPORTED, "grid too large");
   const cudaError_t e = tg::launch_pdl(gated_attention_kernel<D, kBias>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
-                                      C::kSmem, stream, tm_q, tm_k, tm_v, s, gain, scale_log2, cu_seqlens,
+                                      C::kSmem, stream, tm_q, tm_k, tm_v, tm_o, s, gain, scale_log2, cu_seqlens,
                                       cu_seqlens ? int64_t(0) : total, total, n_mblocks, B, Hq, Hkv,
                                       reinterpret_cast<__nv_bfloat16 *>(O), lse, O32, err);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "gated_attention_kernel launch: %s", cudaGetErrorString(e));

@@ -262,6 +262,24 @@ def test_attention_large_bias_and_temperature():
         assert_attn_close(got, oracle.gated_attention(Q, K, V, s, gain, tau))
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_rescale_in_every_key_half(D):
+    # Key scores that climb by ~18 base-2 logit units over every 64 keys, with one jump
+    # of ~140 units: the running max grows past the rescale threshold in the first and
+    # the second half of most KV tiles (the jump alone would overflow fp32 weights if a
+    # rescale were missed or applied to the wrong products).  Rows concentrate on their
+    # last keys, so V is halved as in the other near-one-hot cases.
+    S = 1000
+    Q, K, V, s, gain = _attn_inputs(S, 4, 2, D, 91)
+    V = (V.float() * 0.5).to(torch.bfloat16)
+    s = 0.2 * torch.arange(S, dtype=torch.float32)
+    s[700:] += 100.0
+    gain = torch.ones(4)
+    got = tg.tg_gated_attention(Q.to(DEV), K.to(DEV), V.to(DEV), s.to(DEV), gain.to(DEV), 1.1).float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert_attn_close(got, oracle.gated_attention(Q, K, V, s, gain, 1.1))
+
+
 @pytest.mark.parametrize("tau", [-0.7, 0.0, 1e-3, 2.5])
 def test_attention_temperature_sign_and_zero(tau):
     # tau < 0 flips the order of the logits (largest logit = smallest q.k), tau = 0 leaves
