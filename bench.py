@@ -537,10 +537,26 @@ def cpu_baseline(host, w, S, budget_s: float = 10.0, steps: int = 1):
         oracle.gated_attention(Q, K, V, s, gain, tau, rows=rows)
         times.append(time.perf_counter() - t0)
     el = min(times)
+    full = attention_flops(S, w.hq, w.head_dim)
     return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"fp64 C oracle, gated attention layer 0, last {n_rows} of {S} query rows x {w.hq} heads "
-                      f"(the longest causal rows), {flops:.3e} flops in {el:.2f} s"}
+                      f"(the longest causal rows), {flops:.3e} flops in {el:.2f} s",
+            "rows_per_s": round(n_rows / el, 2),
+            "extrapolated_full_layer_s": round(full / (flops / el), 2),
+            "affinity_cores": len(os.sched_getaffinity(0)), "cpu_model": host_cpu_model()}
+
+
+def host_cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), for the oracle's timing record."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, world, rank):
@@ -573,7 +589,8 @@ def run_reference(args, world, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(world, K, S, w.layers, w.n),
             "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample,
+                             "affinity_cores": len(os.sched_getaffinity(0)), "cpu_model": host_cpu_model()},
             "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
