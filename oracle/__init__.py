@@ -55,12 +55,20 @@ def lib():
         L.orc_linear_rows.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_set_num_threads.argtypes = [i32]
+        L.orc_set_num_threads.restype = None
         _lib = L
     return _lib
 
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Thread count of the oracle's parallel loops from now on (timing only; results are
+    the same for any count)."""
+    lib().orc_set_num_threads(int(n))
 
 
 def _bf16_bits(t: torch.Tensor) -> np.ndarray:

@@ -514,6 +514,18 @@ void orc_linear_rows(const uint16_t *x, int32_t K, const uint16_t *W, int32_t N,
     }
 }
 
+/* Thread count of the following parallel regions (timing on one core, for reporting);
+ * n <= 0 leaves it unchanged.  Results do not depend on it. */
+void orc_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the oracle runs with (for reporting). */
 int orc_num_threads(void)
 {

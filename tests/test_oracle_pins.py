@@ -648,3 +648,25 @@ def test_lse_matches_torch_logsumexp():
     assert np.allclose(oracle.gated_attention_lse(Q, K, s, gain, tau), ref, rtol=1e-12, atol=1e-12)
     rows = [32, 0, 7]
     assert np.allclose(oracle.gated_attention_lse(Q, K, s, gain, tau, rows=rows), ref[rows], rtol=1e-12, atol=1e-12)
+
+
+def test_oracle_results_do_not_depend_on_thread_count():
+    # the timed CPU baseline also runs the oracle on one core; every row is computed by
+    # one thread in a fixed order, so the count cannot change a single bit
+    g = torch.Generator().manual_seed(12)
+    S, Hq, Hkv, D = 70, 4, 2, 16
+    Q = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    K = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    s = torch.randn(S, generator=g)
+    gain = 0.5 + torch.rand(Hq, generator=g)
+    many = oracle.num_threads()
+    ref = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    oracle.set_num_threads(1)
+    try:
+        assert oracle.num_threads() == 1
+        one = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    finally:
+        oracle.set_num_threads(many)
+    assert oracle.num_threads() == many
+    assert np.array_equal(one, ref)
