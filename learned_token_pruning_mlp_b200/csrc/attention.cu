@@ -46,8 +46,10 @@
 //     rescaled in TMEM after P is stored (S_t(j) completing orders this after O_t's
 //     previous product).  Otherwise exponentials are taken against the stale max,
 //     which stays exact in fp32 and loses nothing in bf16.
-//   * The epilogue divides O by the row sum, converts to bf16 and stores the rows;
-//     for training it also stores each row's log-sum-exp (natural log), from which
+//   * The epilogue divides O by the row sum and converts it to bf16; a whole tile is
+//     staged in shared memory (over its finished Q tile) and written by one tensor
+//     store, a partial tile row by row.  For training it also stores each row's
+//     log-sum-exp (natural log), from which
 //     the backward recomputes the probabilities, and optionally the output before its
 //     bf16 rounding (fp32), from which the backward forms dO . O.
 //   * CTAs are ordered heaviest first (the longest causal rows), which the hardware
