@@ -59,3 +59,45 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_zero():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def _bench_module():
+    sys.path.insert(0, ROOT)
+    import bench
+    return bench
+
+
+def test_attention_flops_count_the_visible_pairs():
+    bench = _bench_module()
+    for S in (1, 2, 7, 130):
+        pairs = sum(1 for i in range(S) for j in range(S) if j <= i)
+        assert bench.attention_flops(S, 3, 16) == 4 * 16 * 3 * pairs  # QK^T and PV, 2 flops per multiply-add
+    assert bench.attention_flops(8704, 16, 128) == 310_347_038_720
+
+
+def test_select_path_bytes_at_the_128k_workload():
+    bench = _bench_module()
+    # gate: residual read, W1, b1/W2 (+b2), scores written; top-K: scores + mask read, kept
+    # indices (+count) written; gather: indices, rows read and written, scores gathered
+    assert bench.select_path_bytes(131072, 2048, 256, 8704) == 610_543_110
+
+
+def test_clock_sampler_reads_median_clock_and_reasons():
+    bench = _bench_module()
+
+    class _Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    cs = bench.ClockSampler(0)
+    cs.proc = _Proc()
+    cs.lines = ["0, 1965, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active",
+                "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+                "0, 1900, 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+                "garbage line"]
+    out = cs.stop()
+    assert out["sm_mhz"] == 1900 and out["sm_max_mhz"] == 1965 and out["samples"] == 3
+    assert out["reasons"] == ["sw_power_cap"]
