@@ -198,7 +198,6 @@ def random_scores(n: int, seed: int) -> torch.Tensor:
     return torch.randn(n, generator=_gen(seed, "sel"), dtype=torch.float32)
 
 
-
 def layer_weights(w: Workload, layer: int = 0):
     """Synthetic weights of one pruned attention layer, all bf16:
     W_qkv [(hq + 2 hkv) D, d] ~ N(0, 1/d) (Q rows, then K rows, then V rows),
