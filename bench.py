@@ -41,7 +41,7 @@ METRIC = "gated-attn TFLOP/s & % bf16 peak; gate+topK+gather GB/s & % HBM, N=128
 DATASHEET_HBM_GBS = 8000.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch at
-# S = 8704, from the ncu capture summarised in profiles/attention_qwen3_1p7b_n128k_layer.md.
+# S = 8704, from one ncu capture of the kernel (its summary is kept with the profiles).
 # It is reported only while the kernel sources are the ones that capture measured.
 ATTENTION_TRAFFIC = {"sources_sha1": "743548f20766cd6c49c4c9f7fb5019e1ff6048a2", "bytes_per_launch": 72093184 + 9845248}
 

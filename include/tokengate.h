@@ -22,13 +22,26 @@
  *     CUDA graph.
  *   - The return value reports errors that the host can detect (shapes,
  *     alignment, null pointers, unsupported sizes, launch failures).  When it
- *     is not TG_OK nothing was launched; tg_last_error_detail() describes it.
+ *     is not TG_OK nothing was launched, with one exception: a call that
+ *     launches several kernels (tg_select_topk_varlen, tg_select_fused, the
+ *     backward) and whose second or later launch fails returns TG_ERR_CUDA with
+ *     the earlier kernels already queued; its outputs and workspace are then
+ *     undefined.  tg_last_error_detail() describes the error.
  *   - Conditions only the device can see (an index out of range, a budget
  *     above the document length, a full output, a bounded wait that ran out)
  *     set bits in a sticky per-device status word and never trap.  Read and
  *     clear it with tg_get_device_error().
  *   - Calls on different streams may run concurrently; they share only the
- *     status word, whose bits are OR-ed.
+ *     status word, whose bits are OR-ed.  Exception: every
+ *     tg_gated_attention_backward_noalloc call on a device uses the same static
+ *     scratch array, so those calls must be ordered on the device (one stream,
+ *     or streams that wait on each other).
+ *   - Host threads may call the library concurrently.  Per-device set-up (kernel
+ *     attributes, the device addresses of the status word and of the static
+ *     scratch) is done by the first call on each device and kept for the life of
+ *     the process, so a device reset (cudaDeviceReset) invalidates it: do not use
+ *     the library on a device after resetting that device.
+ *   - Every call opens an NVTX range named after it on the calling host thread.
  */
 #ifndef TOKENGATE_H
 #define TOKENGATE_H

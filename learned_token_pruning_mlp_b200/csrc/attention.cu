@@ -548,10 +548,8 @@ tg_status launch_kernel(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, c
     if (!tg::encode_tmap(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return TG_ERR_CUDA;
   }
-  static bool configured[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  static tg::PerDevice configured;
+  const tg_status setup = tg::once_per_device(configured, [&](int) -> tg_status {
     const cudaError_t e = cudaFuncSetAttribute(gated_attention_kernel<D, kBias>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -562,8 +560,9 @@ tg_status launch_kernel(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, c
     if (fa.numRegs != 168)
       return tg::fail(TG_ERR_UNSUPPORTED, "gated_attention_kernel built with %d registers per thread; the register "
                       "split needs 168", fa.numRegs);
-    configured[dev] = true;
-  }
+    return TG_OK;
+  });
+  if (setup != TG_OK) return setup;
   const float scale_log2 = tau / std::sqrt(static_cast<float>(D)) * kLog2e;
   const int n_mblocks = static_cast<int>((max_seqlen + 2 * kBM - 1) / (2 * kBM));
   const int64_t grid = static_cast<int64_t>(n_mblocks) * Hq * B;
@@ -610,7 +609,7 @@ tg_status validate(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const 
 extern "C" tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
                                         const float *gain, float tau, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
                                         tg_bf16 *O, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   tg_status st = validate(Q, Kc, V, s, gain, tau, S, Hq, Hkv, D, O);
   if (st != TG_OK || S == 0) return st;
   uint32_t *err = tg::device_error_word();
@@ -623,7 +622,7 @@ extern "C" tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, con
 extern "C" tg_status tg_gated_attention_train(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
                                               const float *gain, float tau, int64_t S, int32_t Hq, int32_t Hkv,
                                               int32_t D, tg_bf16 *O, float *lse, float *O32, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   tg_status st = validate(Q, Kc, V, s, gain, tau, S, Hq, Hkv, D, O);
   if (st != TG_OK || S == 0) return st;
   if (!lse) return tg::fail(TG_ERR_INVALID_ARG, "lse is NULL");
@@ -639,7 +638,7 @@ extern "C" tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *
                                                const float *gain, float tau, const int32_t *cu_seqlens, int32_t B,
                                                int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
                                                tg_bf16 *O, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (B < 0) return tg::fail(TG_ERR_INVALID_ARG, "B must be >= 0");
   if (max_seqlen < 0 || max_seqlen > total) return tg::fail(TG_ERR_INVALID_ARG, "max_seqlen must be in [0, total]");
   if (B > 0 && !cu_seqlens) return tg::fail(TG_ERR_INVALID_ARG, "cu_seqlens is NULL");

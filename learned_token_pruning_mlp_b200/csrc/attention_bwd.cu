@@ -432,10 +432,8 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
   if (!tmap3(&tm_q, Q, D, Hq, S) || !tmap3(&tm_k, Kc, D, Hkv, S) || !tmap3(&tm_v, V, D, Hkv, S) ||
       !tmap3(&tm_do, dO, D, Hq, S))
     return TG_ERR_CUDA;
-  static bool configured[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  static tg::PerDevice configured;
+  const tg_status setup = tg::once_per_device(configured, [&](int) -> tg_status {
     const cudaError_t e =
         cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -446,8 +444,9 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
     if (fa.numRegs != 168)
       return tg::fail(TG_ERR_UNSUPPORTED, "attn_bwd_kernel built with %d registers per thread; the register split "
                       "needs 168", fa.numRegs);
-    configured[dev] = true;
-  }
+    return TG_OK;
+  });
+  if (setup != TG_OK) return setup;
   const int64_t prep_warps = S_pad * Hq;  // below 2^31 (checked by the caller)
   const unsigned prep_grid = static_cast<unsigned>((prep_warps + 7) / 8);
   cudaError_t e = tg::launch_pdl(attn_bwd_prep_kernel<D>, dim3(prep_grid), dim3(256), 0, stream,
@@ -491,7 +490,7 @@ extern "C" tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16
                                                  int32_t Hq,
                                                  int32_t Hkv, int32_t D, float *ds, float *dgain, float *dtau,
                                                  void *workspace, size_t workspace_size, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (S < 0) return tg::fail(TG_ERR_INVALID_ARG, "S must be >= 0");
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return tg::fail(TG_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv");
   if (D != 64 && D != 128) return tg::fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
@@ -526,7 +525,7 @@ extern "C" tg_status tg_gated_attention_backward_noalloc(const tg_bf16 *Q, const
                                                          const float *lse, int64_t S, int32_t Hq, int32_t Hkv,
                                                          int32_t D, float *ds, float *dgain, float *dtau,
                                                          tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (S < 0) return tg::fail(TG_ERR_INVALID_ARG, "S must be >= 0");
   if (Hq <= 0) return tg::fail(TG_ERR_INVALID_ARG, "Hq must be positive");
   if (padded_rows(S) * Hq > (int64_t(1) << 31) - 1) return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
@@ -538,19 +537,25 @@ extern "C" tg_status tg_gated_attention_backward_noalloc(const tg_bf16 *Q, const
                     static_cast<long long>(S), Hq, need, kStaticScratchBytes);
   void *scratch = nullptr;
   if (S > 0) {
-    // the array's address on the current device, looked up once per device
-    static void *cached[64];
+    // The array's device address (host code may not use the symbol itself), looked up
+    // by the first call on each device with that device current, under the library's
+    // set-up lock, and read without the lock afterwards.
+    static std::atomic<void *> addr[tg::kMaxDevices];
+    static tg::PerDevice looked_up;
     int dev = 0;
-    const cudaError_t ed = cudaGetDevice(&dev);
-    if (ed != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(ed));
-    if (dev >= 0 && dev < 64 && cached[dev]) {
-      scratch = cached[dev];
-    } else {
-      const cudaError_t e = cudaGetSymbolAddress(&scratch, g_bwd_scratch);
-      if (e != cudaSuccess || !scratch)
-        return tg::fail(TG_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-      if (dev >= 0 && dev < 64) cached[dev] = scratch;
-    }
+    const tg_status st = tg::once_per_device(
+        looked_up,
+        [&](int d) -> tg_status {
+          void *p = nullptr;
+          const cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+          if (e != cudaSuccess || !p)
+            return tg::fail(TG_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+          addr[d].store(p, std::memory_order_relaxed);  // published by the set-up flag's release
+          return TG_OK;
+        },
+        &dev);
+    if (st != TG_OK) return st;
+    scratch = addr[dev].load(std::memory_order_relaxed);
   }
   return tg_gated_attention_backward(Q, Kc, V, s, gain, tau, O, O32, dO, lse, S, Hq, Hkv, D, ds, dgain, dtau, scratch,
                                      kStaticScratchBytes, stream);

@@ -275,15 +275,14 @@ tg_status tg::gate_score_hist(const tg_bf16 *hidden, int64_t n, int32_t d, const
   while (tmem_cols < 2u * static_cast<uint32_t>(h)) tmem_cols <<= 1;
 
   const size_t smem = smem_bytes(h);
-  static bool configured[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  static tg::PerDevice configured;
+  const tg_status setup = tg::once_per_device(configured, [&](int) -> tg_status {
     const cudaError_t e = cudaFuncSetAttribute(gate_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem_bytes(kMaxH)));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    configured[dev] = true;
-  }
+    return TG_OK;
+  });
+  if (setup != TG_OK) return setup;
   const cudaError_t e = tg::launch_pdl(gate_score_kernel, dim3(static_cast<unsigned>(gate_grid(n))), dim3(kThreads), smem,
                                       static_cast<cudaStream_t>(stream), tm_x, tm_w,
                                       reinterpret_cast<const __nv_bfloat16 *>(b1),
@@ -296,6 +295,6 @@ tg_status tg::gate_score_hist(const tg_bf16 *hidden, int64_t n, int32_t d, const
 
 extern "C" tg_status tg_gate_score(const tg_bf16 *hidden, int64_t n, int32_t d, const tg_bf16 *W1, const tg_bf16 *b1,
                                    const tg_bf16 *W2, const tg_bf16 *b2, int32_t h, float *scores, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   return tg::gate_score_hist(hidden, n, d, W1, b1, W2, b2, h, scores, nullptr, nullptr, stream);
 }

@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(
 extern "C" tg_status tg_gather(const tg_bf16 *hidden, int64_t n, int32_t d, const int32_t *kept_idx,
                                int64_t n_rows, const int32_t *n_kept, tg_bf16 *hidden_k, const float *scores,
                                float *s_k, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (n < 0 || n_rows < 0) return tg::fail(TG_ERR_INVALID_ARG, "negative n or n_rows");
   if (d <= 0 || d % 8 != 0) return tg::fail(TG_ERR_INVALID_ARG, "d must be a positive multiple of 8 (got %d)", d);
   if (d > 16384) return tg::fail(TG_ERR_UNSUPPORTED, "d above 16384 (got %d)", d);

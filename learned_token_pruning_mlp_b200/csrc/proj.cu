@@ -380,10 +380,8 @@ tg_status launch_proj(const tg_bf16 *x, int64_t M, int32_t K, const tg_bf16 *W, 
     if (!tg::encode_tmap(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return TG_ERR_CUDA;
   }
-  static bool configured[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  static tg::PerDevice configured;
+  const tg_status setup = tg::once_per_device(configured, [&](int) -> tg_status {
     const cudaError_t e =
         cudaFuncSetAttribute(proj_gemm_kernel<kHD>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -396,8 +394,9 @@ tg_status launch_proj(const tg_bf16 *x, int64_t M, int32_t K, const tg_bf16 *W, 
         return tg::fail(TG_ERR_UNSUPPORTED, "%s built with %d registers per thread; the warpgroup register split "
                         "needs 168", name, fa.numRegs);
     }
-    configured[dev] = true;
-  }
+    return TG_OK;
+  });
+  if (setup != TG_OK) return setup;
   const int64_t tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kBN - 1) / kBN);
   if (tiles > 0x7FFFFFFF) return tg::fail(TG_ERR_UNSUPPORTED, "%s: more than 2^31 - 1 output tiles", name);
   const int64_t pairs = std::min<int64_t>(tiles, tg::sm_count() / 2);
@@ -411,7 +410,7 @@ tg_status launch_proj(const tg_bf16 *x, int64_t M, int32_t K, const tg_bf16 *W, 
 
 extern "C" tg_status tg_linear(const tg_bf16 *x, int64_t M, int32_t K, const tg_bf16 *W, int32_t N,
                                const tg_bf16 *residual, tg_bf16 *y, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (M < 0 || K <= 0 || N <= 0) return tg::fail(TG_ERR_INVALID_ARG, "M >= 0, K > 0, N > 0 required");
   if (K % 8 != 0) return tg::fail(TG_ERR_UNSUPPORTED, "K must be a multiple of 8 (got %d)", K);
   if (N % 32 != 0) return tg::fail(TG_ERR_UNSUPPORTED, "N must be a multiple of 32 (got %d)", N);
@@ -430,7 +429,7 @@ extern "C" tg_status tg_qkv_rope(const tg_bf16 *hidden, int64_t S, int32_t d, co
                                  const int32_t *positions, double rope_base, const tg_bf16 *q_norm,
                                  const tg_bf16 *k_norm, float eps, int32_t Hq, int32_t Hkv, int32_t D, tg_bf16 *Q,
                                  tg_bf16 *Kc, tg_bf16 *V, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (S < 0 || d <= 0) return tg::fail(TG_ERR_INVALID_ARG, "S >= 0 and d > 0 required");
   if (d % 8 != 0) return tg::fail(TG_ERR_UNSUPPORTED, "d must be a multiple of 8 (got %d)", d);
   if (D != 64 && D != 128) return tg::fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);

@@ -17,7 +17,6 @@ namespace tg {
 namespace {
 thread_local char t_detail[512];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 uint32_t *g_word_addr[kMaxDevices];
 int g_sms[kMaxDevices];
@@ -36,6 +35,11 @@ int current_device() {
 }  // namespace
 
 void clear_detail() { t_detail[0] = 0; }
+
+std::mutex &setup_mutex() {
+  static std::mutex mu;
+  return mu;
+}
 
 tg_status fail(tg_status st, const char *fmt, ...) {
   va_list ap;
@@ -155,7 +159,7 @@ const char *tg_status_string(tg_status st) {
 const char *tg_last_error_detail(void) { return tg::t_detail; }
 
 tg_status tg_get_device_error(tg_stream stream, uint32_t *bits) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (!bits) return tg::fail(TG_ERR_INVALID_ARG, "bits is NULL");
   *bits = 0;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
@@ -171,7 +175,7 @@ tg_status tg_get_device_error(tg_stream stream, uint32_t *bits) {
 }
 
 tg_status tg_probe_wait_timeout(int64_t limit_ns, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (limit_ns <= 0 || limit_ns > 2000000000LL)
     return tg::fail(TG_ERR_INVALID_ARG, "limit_ns must be in (0, 2e9]");
   uint32_t *err = tg::device_error_word();

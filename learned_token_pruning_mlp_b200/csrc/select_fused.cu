@@ -27,7 +27,7 @@ extern "C" tg_status tg_select_fused(const tg_bf16 *hidden, int64_t n, int32_t d
                                      const uint8_t *doc_mask, int64_t k, float *scores, int32_t *kept_idx,
                                      int64_t cap, int32_t *n_kept, tg_bf16 *hidden_k, float *s_k, int64_t n_rows,
                                      void *workspace, size_t workspace_bytes, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
   if (n_rows < 0) return tg::fail(TG_ERR_INVALID_ARG, "n_rows must be >= 0");
   if (n_rows > cap) return tg::fail(TG_ERR_INVALID_ARG, "n_rows must not exceed cap");

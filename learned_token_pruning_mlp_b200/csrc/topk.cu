@@ -492,7 +492,7 @@ int64_t chunk_of(int64_t len) { return ((len + kCluster - 1) / kCluster + kItems
 
 extern "C" tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask, int64_t n, int64_t k,
                                     int32_t *kept_idx, int64_t cap, int32_t *n_kept, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
   if (k < 0) return tg::fail(TG_ERR_INVALID_ARG, "k must be >= 0");
   if (cap < 0) return tg::fail(TG_ERR_INVALID_ARG, "cap must be >= 0");
@@ -547,7 +547,7 @@ tg_status tg::select_topk_hist(const float *scores, const uint8_t *doc_mask, int
 
 extern "C" tg_status tg_select_random_k(const uint8_t *doc_mask, int64_t n, int64_t k, uint64_t seed,
                                         int32_t *kept_idx, int64_t cap, int32_t *n_kept, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
   if (k < 0) return tg::fail(TG_ERR_INVALID_ARG, "k must be >= 0");
   if (cap < 0) return tg::fail(TG_ERR_INVALID_ARG, "cap must be >= 0");
@@ -575,7 +575,7 @@ extern "C" tg_status tg_select_random_k(const uint8_t *doc_mask, int64_t n, int6
 extern "C" tg_status tg_select_topk_sweep(const float *scores, const uint8_t *doc_mask, int64_t n,
                                           const int32_t *ks, int32_t m, int32_t *kept_idx, int64_t stride,
                                           int32_t *n_kept, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (n < 0 || n > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "n must be in [0, 2^31) (got %lld)", (long long)n);
   if (m < 0 || m > 65535) return tg::fail(TG_ERR_INVALID_ARG, "the number of budgets must be in [0, 65535]");
   if (stride < 0 || (m > 0 && stride > 0x7FFFFFFFLL / m))
@@ -606,7 +606,7 @@ extern "C" tg_status tg_select_topk_sweep(const float *scores, const uint8_t *do
 extern "C" tg_status tg_select_topk_varlen(const float *scores, const uint8_t *doc_mask, const int32_t *cu_seqlens,
                                            int32_t B, int64_t total, const int32_t *k_per_seq, int64_t max_seqlen,
                                            int32_t *kept_idx, int64_t cap, int32_t *cu_kept, tg_stream stream) {
-  tg::clear_detail();
+  TG_API_ENTRY();
   if (B < 0) return tg::fail(TG_ERR_INVALID_ARG, "B must be >= 0");
   if (total < 0 || total > 0x7FFFFFFFLL) return tg::fail(TG_ERR_INVALID_ARG, "total must be in [0, 2^31)");
   if (max_seqlen < 0 || max_seqlen > total) return tg::fail(TG_ERR_INVALID_ARG, "max_seqlen must be in [0, total]");
