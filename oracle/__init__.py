@@ -39,7 +39,7 @@ def lib():
         L.orc_select_topk.restype = i64
         L.orc_gather.argtypes = [vp, i32, vp, i64, vp, vp, vp]
         L.orc_gather.restype = None
-        L.orc_gated_attention_rows.argtypes = [vp, vp, vp, vp, vp, f64, i64, i32, i32, i32, vp, i64, vp]
+        L.orc_gated_attention_rows.argtypes = [vp, vp, vp, vp, vp, f64, i64, i32, i32, i32, vp, i64, vp, vp]
         L.orc_gated_attention_rows.restype = None
         L.orc_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
         L.orc_splitmix64.restype = ctypes.c_uint64
@@ -161,9 +161,14 @@ def gather(hidden, kept, scores=None):
 
 
 # --------------------------------------------------------------------------- attention
-def gated_attention(Q, K, V, s, gain, tau: float, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+def gated_attention(Q, K, V, s, gain, tau: float, rows: Optional[Sequence[int]] = None,
+                    return_spread: bool = False):
     """O[i,h] = sum_{j<=i} softmax_j(tau*Q_ih.K_jg/sqrt(D) + gain_h*s_j) V_jg, g = h // (Hq/Hkv).
-    Returns fp64 [len(rows), Hq, D] (all rows when ``rows`` is None)."""
+    Returns fp64 [len(rows), Hq, D] (all rows when ``rows`` is None).  With
+    ``return_spread`` also returns spread[i,h,c] = sum_j softmax_j |V_jg[c] - O_ih[c]|,
+    the weighted mean absolute deviation of the value rows: a bound on how far
+    relative weight errors move the output, used to size tolerances (not part of
+    the method)."""
     S, Hq, D = Q.shape
     Hkv = K.shape[1]
     qb, kb, vb = _bf16_bits(Q), _bf16_bits(K), _bf16_bits(V)
@@ -171,27 +176,35 @@ def gated_attention(Q, K, V, s, gain, tau: float, rows: Optional[Sequence[int]] 
     gv = _np(gain, np.float32)
     r = np.arange(S, dtype=np.int64) if rows is None else _np(rows, np.int64)
     out = np.empty((len(r), Hq, D), dtype=np.float64)
+    spread = np.empty((len(r), Hq, D), dtype=np.float64) if return_spread else None
     lib().orc_gated_attention_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(sv), _ptr(gv), float(tau),
-                                   S, Hq, Hkv, D, _ptr(r), len(r), _ptr(out))
-    return out
+                                   S, Hq, Hkv, D, _ptr(r), len(r), _ptr(out),
+                                   _ptr(spread) if return_spread else None)
+    return (out, spread) if return_spread else out
 
 
 def gated_attention_varlen(Q, K, V, s, gain, tau: float, cu_seqlens: Sequence[int],
-                           rows: Optional[Sequence[int]] = None) -> np.ndarray:
+                           rows: Optional[Sequence[int]] = None, return_spread: bool = False):
     """Packed requests: each segment [cu[b], cu[b+1]) attends causally within itself only.
-    ``rows`` are packed row indices (all rows when None); returns fp64 [len(rows), Hq, D]."""
+    ``rows`` are packed row indices (all rows when None); returns fp64 [len(rows), Hq, D]
+    (and the spread, as in ``gated_attention``)."""
     cu = [int(x) for x in cu_seqlens]
     S, Hq, D = Q.shape
     rows_all = np.arange(S, dtype=np.int64) if rows is None else _np(rows, np.int64)
     out = np.empty((len(rows_all), Hq, D), dtype=np.float64)
+    spread = np.empty((len(rows_all), Hq, D), dtype=np.float64) if return_spread else None
     for b in range(len(cu) - 1):
         lo, hi = cu[b], cu[b + 1]
         sel = np.nonzero((rows_all >= lo) & (rows_all < hi))[0]
         if len(sel) == 0:
             continue
-        out[sel] = gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], _np(s, np.float32)[lo:hi], gain, tau,
-                                   rows=rows_all[sel] - lo)
-    return out
+        res = gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], _np(s, np.float32)[lo:hi], gain, tau,
+                              rows=rows_all[sel] - lo, return_spread=return_spread)
+        if return_spread:
+            out[sel], spread[sel] = res
+        else:
+            out[sel] = res
+    return (out, spread) if return_spread else out
 
 
 def gated_attention_lse(Q, K, s, gain, tau: float, rows: Optional[Sequence[int]] = None) -> np.ndarray:

@@ -239,11 +239,18 @@ void orc_gather(const uint16_t *hidden, int32_t d, const int32_t *kept, int64_t 
  * Q: bf16 [S, Hq, D]; K, V: bf16 [S, Hkv, D]; s: fp32 [S]; gain: fp32 [Hq].
  * Only the rows listed in ``rows`` are computed (all rows for a full run);
  * O: double [n_rows, Hq, D].
+ *
+ * spread (NULL to skip): double [n_rows, Hq, D], the mean absolute deviation of
+ * the value rows under the row's softmax weights,
+ *     spread[i,h,c] = sum_j softmax_j(l_i.) |V[j,g,c] - O[i,h,c]|.
+ * It is not part of the method: it measures how far a perturbation of the weights
+ * can move the output (relative weight errors of at most e move O[i,h,c] by at
+ * most about 2 e spread[i,h,c]), which the tests use to size their tolerance.
  * ------------------------------------------------------------------------ */
 void orc_gated_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                               const float *s, const float *gain, double tau,
                               int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
-                              const int64_t *rows, int64_t n_rows, double *O)
+                              const int64_t *rows, int64_t n_rows, double *O, double *spread)
 {
     const int32_t group = Hq / Hkv;
     const double inv_sqrt_d = 1.0 / sqrt((double)D);
@@ -284,6 +291,15 @@ void orc_gated_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16
                 for (int32_t c = 0; c < D; ++c) o[c] += p * bf16_value(vj[c]);
             }
             for (int32_t c = 0; c < D; ++c) o[c] /= denom;
+            if (spread) {
+                double *sp = spread + ((size_t)r * Hq + hh) * D;
+                for (int32_t c = 0; c < D; ++c) sp[c] = 0.0;
+                for (int64_t j = 0; j <= i; ++j) {
+                    const double w = exp(l[j] - m) / denom;
+                    const uint16_t *vj = V + ((size_t)j * Hkv + g) * D;
+                    for (int32_t c = 0; c < D; ++c) sp[c] += w * fabs(bf16_value(vj[c]) - o[c]);
+                }
+            }
         }
         free(q);
         free(l);

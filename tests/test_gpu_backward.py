@@ -35,6 +35,7 @@ import torch
 
 import oracle
 import learned_token_pruning_mlp_b200 as tg
+from test_gpu_parity import check_attention
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -174,6 +175,20 @@ def test_lse_matches_oracle_and_forward_unchanged():
     assert torch.equal(O32.to(torch.bfloat16), O)  # O is the bf16 rounding of O32
     ref = oracle.gated_attention_lse(Q, K, s, gain, 1.1)
     assert np.max(np.abs(lse.cpu().numpy() - ref)) <= 4e-3
+    # both outputs of the training forward within the forward's rounding budget (the fp32
+    # output without the bf16 output rounding)
+    check_attention(O.float().cpu().numpy(), Q, K, V, s, gain, 1.1)
+    check_attention(O32.cpu().numpy(), Q, K, V, s, gain, 1.1, fp32_out=True)
+
+
+def test_train_forward_varied_shapes_within_budget():
+    for S, Hq, Hkv, D, tau in ((1000, 4, 2, 64, -0.7), (257, 8, 2, 128, 2.5)):
+        Q, K, V, dO, s, gain = _case(S, Hq, Hkv, D, S + D)
+        d = [t.to(DEV) for t in (Q, K, V, s, gain)]
+        O, lse, O32 = tg.tg_gated_attention_train(d[0], d[1], d[2], d[3], d[4], tau)
+        check_attention(O.float().cpu().numpy(), Q, K, V, s, gain, tau)
+        check_attention(O32.cpu().numpy(), Q, K, V, s, gain, tau, fp32_out=True)
+    assert tg.tg_get_device_error() == 0
 
 
 def test_backward_is_deterministic_and_overwrites_outputs():

@@ -9,7 +9,7 @@ is checked against the fp64 oracle:
   * gated attention on a row sample (all heads) over the rows the oracle kept;
   * the all-GPU chain (GPU scores -> GPU top-K -> GPU gather) for the properties the
     article fixes: |kept| = K + question length, every question token kept, ascending.
-Tolerances are the ones of tests/test_gpu_parity.py.
+Tolerances are the ones of the parity tests (test_gpu_parity.py).
 """
 import numpy as np
 import pytest
@@ -18,7 +18,7 @@ import torch
 import oracle
 import learned_token_pruning_mlp_b200 as tg
 from learned_token_pruning_mlp_b200 import workloads as W
-from test_gpu_parity import assert_attn_close, assert_gate_close
+from test_gpu_parity import assert_gate_close, check_attention
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -106,7 +106,7 @@ def test_full_size_path(name, K):
     gain, tau = W.attention_params(w)
     O = tg.tg_gated_attention(Q.to(DEV), Kc.to(DEV), V.to(DEV), torch.as_tensor(ref_sk).to(DEV), gain.to(DEV), tau)
     arows = oracle.sampled_rows(S, seed=S, head=64, tail=64, rand=128)
-    assert_attn_close(O.float().cpu().numpy()[arows], oracle.gated_attention(Q, Kc, V, ref_sk, gain, tau, rows=arows))
+    check_attention(O.float().cpu().numpy()[arows], Q, Kc, V, ref_sk, gain, tau, rows=arows)
     bits = tg.tg_get_device_error()
     assert bits & ~tg.TG_DEVERR_K_GT_NDOC == 0
 
@@ -150,6 +150,5 @@ def test_full_size_ragged_batch():
         arows += list(range(lo, min(lo + 32, hi))) + list(range(max(lo, hi - 32), hi))
         arows += list(rng.choice(np.arange(lo, hi), size=min(32, hi - lo), replace=False))
     arows = np.unique(np.asarray(arows, dtype=np.int64))
-    assert_attn_close(O.float().cpu().numpy()[arows],
-                      oracle.gated_attention_varlen(Q, Kc, V, ref_sk, gain, tau, ref_cu, rows=arows))
+    check_attention(O.float().cpu().numpy()[arows], Q, Kc, V, ref_sk, gain, tau, rows=arows, cu=ref_cu)
     assert tg.tg_get_device_error() == 0

@@ -210,3 +210,52 @@ def test_backward_pins_reject_planted_mistakes():
     assert not passes(gain_in_ds=False)    # score gradient without the head's gain
     assert not passes(sqrt_d=False)        # temperature gradient without 1/sqrt(D)
     assert not passes(causal=False)        # keys after the query counted
+
+
+def _spread_variant(Q, K, V, s, gain, tau, *, mode="ok"):
+    """A CPU copy of the spread (sum_j w_j |V_j - O|) with one planted mistake."""
+    q, kk, v = Q.double().numpy(), K.double().numpy(), V.double().numpy()
+    sv, gv = np.asarray(s, np.float64), np.asarray(gain, np.float64)
+    S, Hq, D = q.shape
+    Hkv = kk.shape[1]
+    out = np.empty((S, Hq, D))
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        L = tau * (q[:, h] @ kk[:, g].T) / math.sqrt(D) + gv[h] * sv[None, :]
+        L = np.where(np.tril(np.ones((S, S), bool)), L, -np.inf)
+        P = np.exp(L - L.max(1, keepdims=True))
+        if mode != "unnormalised":
+            P /= P.sum(1, keepdims=True)
+        O = P @ v[:, g] if mode != "unnormalised" else (P @ v[:, g]) / P.sum(1, keepdims=True)
+        for c in range(D):
+            dev = v[None, :, g, c] - O[:, None, c]
+            if mode == "no_abs":
+                out[:, h, c] = (P * dev).sum(1)
+            elif mode == "abs_v":
+                out[:, h, c] = (P * np.abs(v[None, :, g, c])).sum(1)
+            else:
+                out[:, h, c] = (P * np.abs(dev)).sum(1)
+    return out
+
+
+def test_spread_pins_reject_planted_mistakes():
+    """The two-key identity and row 0 (the spread pins) reject a spread without the
+    absolute value, one of |V| instead of |V - O|, and one with unnormalised weights."""
+    Q, K, V, s, gain = _attn_case(12, 2, 1, 8, 77)
+    o = oracle.gated_attention(Q, K, V, s, gain, 1.1)
+    v = V.double().numpy()
+
+    def pins_hold(sp):
+        if not np.allclose(sp[0], 0.0, atol=1e-12):
+            return False
+        for h in range(2):
+            a, b = v[0, 0], v[1, 0]
+            want = 2 * np.abs(o[1, h] - b) * np.abs(a - o[1, h]) / np.abs(a - b)
+            if not np.allclose(sp[1, h], want, rtol=1e-9, atol=1e-12):
+                return False
+        return True
+
+    assert pins_hold(_spread_variant(Q, K, V, s, gain, 1.1))
+    assert pins_hold(oracle.gated_attention(Q, K, V, s, gain, 1.1, return_spread=True)[1])
+    for mode in ("no_abs", "abs_v", "unnormalised"):
+        assert not pins_hold(_spread_variant(Q, K, V, s, gain, 1.1, mode=mode)), mode

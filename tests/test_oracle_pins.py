@@ -349,6 +349,64 @@ def test_attention_varlen_is_block_diagonal():
         np.testing.assert_array_equal(o[lo:hi], oracle.gated_attention(Q[lo:hi], K[lo:hi], V[lo:hi], s[lo:hi], gain, 1.1))
 
 
+# ------------------------------------------------------------ spread (tolerance sizing)
+def test_attention_spread_hand_worked():
+    """spread[i,c] = sum_j w_ij |V_jc - O_ic| by hand on the fixture's cases.  'uniform':
+    row 1 averages V0 = (1, 2) and V1 = (3, -2): O = (2, 0), spread = (1, 2); row 2 averages
+    three rows: O = (1, 2), spread = ((0 + 2 + 2) / 3, (0 + 4 + 4) / 3).  'ln3_bias': row 1
+    weights 1/4, 3/4: O = (2.5, -1), spread = 2 (1/4)(3/4) |V0 - V1| = (0.75, 1.5); row 2
+    weights 0.2, 0.6, 0.2: O = (1.8, 0.4), spread = (0.16 + 0.72 + 0.56, 0.32 + 1.44 + 1.12)."""
+    with open(os.path.join(GOLDEN, "attention_worked.json")) as f:
+        ex = {e["name"]: e for e in json.load(f)["examples"]}
+    expected = {"uniform": [[0.0, 0.0], [1.0, 2.0], [4.0 / 3.0, 8.0 / 3.0]],
+                "ln3_bias": [[0.0, 0.0], [0.75, 1.5], [1.44, 2.88]]}
+    for name, want in expected.items():
+        e = ex[name]
+        Q, K, V = (_bf16(e[k])[:, None, :] for k in ("Q", "K", "V"))
+        o, sp = oracle.gated_attention(Q, K, V, np.asarray(e["s"], np.float32), np.asarray([e["gain"]], np.float32),
+                                       e["tau"], return_spread=True)
+        np.testing.assert_allclose(o[:, 0, :], np.asarray(e["O"]), rtol=0, atol=max(e["tol"], 1e-15))
+        np.testing.assert_allclose(sp[:, 0, :], np.asarray(want), rtol=0, atol=max(4 * e["tol"], 1e-14), err_msg=name)
+
+
+def test_attention_spread_invariants():
+    """Row 0 sees one key (spread 0); with two visible keys the weights follow from O
+    itself (w0 = (O - V1) / (V0 - V1)), so spread = 2 |O - V1| |V0 - O| / |V0 - V1|; the
+    spread does not move when V is shifted and scales with V; constant V rows give 0; it
+    never exceeds the largest deviation of a visible V row; O is unchanged by asking."""
+    Q, K, V, s, gain = _attn_case(60, 4, 2, 16, 131)
+    # V on a 1/8 grid in [-4, 4) so that V + 2 and 2 V are exact in bf16
+    g = torch.Generator().manual_seed(7)
+    V = (torch.randint(-32, 32, V.shape, generator=g).float() / 8).to(torch.bfloat16)
+    o, sp = oracle.gated_attention(Q, K, V, s, gain, 1.1, return_spread=True)
+    np.testing.assert_array_equal(o, oracle.gated_attention(Q, K, V, s, gain, 1.1))
+    assert np.all(sp >= 0)
+    np.testing.assert_allclose(sp[0], 0.0, atol=1e-15)
+    v = V.double().numpy()
+    for h in range(4):
+        a, b = v[0, h // 2], v[1, h // 2]
+        ok = np.abs(a - b) > 0
+        want = 2 * np.abs(o[1, h] - b) * np.abs(a - o[1, h]) / np.where(ok, np.abs(a - b), 1.0)
+        np.testing.assert_allclose(sp[1, h][ok], want[ok], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(sp[1, h][~ok], 0.0, atol=1e-12)
+        for i in (5, 33, 59):
+            dev = np.abs(v[: i + 1, h // 2] - o[i, h]).max(axis=0)
+            assert np.all(sp[i, h] <= dev + 1e-12)
+    _, sp_shift = oracle.gated_attention(Q, K, (V.float() + 2).to(torch.bfloat16), s, gain, 1.1, return_spread=True)
+    np.testing.assert_allclose(sp_shift, sp, rtol=1e-9, atol=1e-12)
+    _, sp_scale = oracle.gated_attention(Q, K, (V.float() * 2).to(torch.bfloat16), s, gain, 1.1, return_spread=True)
+    np.testing.assert_allclose(sp_scale, 2 * sp, rtol=1e-9, atol=1e-12)
+    Vc = torch.full_like(V, 1.5)
+    _, sp_const = oracle.gated_attention(Q, K, Vc, s, gain, 1.1, return_spread=True)
+    np.testing.assert_allclose(sp_const, 0.0, atol=1e-12)
+    # rows, varlen and the full run agree
+    rows = np.array([0, 7, 59])
+    o_r, sp_r = oracle.gated_attention(Q, K, V, s, gain, 1.1, rows=rows, return_spread=True)
+    np.testing.assert_array_equal(sp_r, sp[rows])
+    _, sp_v = oracle.gated_attention_varlen(Q, K, V, s, gain, 1.1, [0, 60], return_spread=True)
+    np.testing.assert_array_equal(sp_v, sp)
+
+
 # ============================================================================ pipeline
 def test_pruned_tokens_never_influence_outputs():
     """Layers above the gate see only kept tokens and keep no KV for pruned ones: poisoning
