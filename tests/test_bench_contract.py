@@ -101,3 +101,22 @@ def test_clock_sampler_reads_median_clock_and_reasons():
     out = cs.stop()
     assert out["sm_mhz"] == 1900 and out["sm_max_mhz"] == 1965 and out["samples"] == 3
     assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_attention_algorithmic_bytes_at_the_128k_layer():
+    bench = _bench_module()
+    read, write = bench.attention_bytes(8704, 16, 8, 128)
+    # Q (16 heads) + K + V (8 heads each) in bf16, the key scores and the gains read once; O written once
+    assert read == (16 + 8 + 8) * 128 * 2 * 8704 + 4 * 8704 + 4 * 16 == 71_338_048
+    assert write == 16 * 128 * 2 * 8704 == 35_651_584
+
+
+def test_sweep_covers_every_workload_budget():
+    bench = _bench_module()
+    from learned_token_pruning_mlp_b200 import workloads as W
+    for name, w in W.WORKLOADS.items():
+        listed = sorted(k for nm, k in bench.SWEEP if nm == name)
+        if w.varlen:
+            assert listed == [None]          # one line for the packed batch (per-request budgets)
+        elif name != "tiny_n512":            # the tiny case is a parity case, not a bench line
+            assert listed == sorted(w.budgets), name
