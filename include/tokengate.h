@@ -272,6 +272,16 @@ tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const t
                                     int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
                                     tg_bf16 *O, tg_stream stream);
 
+/* The training forward of a packed ragged batch: the outputs of
+ * tg_gated_attention_varlen plus lse and O32 as in tg_gated_attention_train, at the
+ * packed rows (lse [total, Hq], O32 [total, Hq, D] or NULL).  Rows outside every
+ * request are left untouched. */
+tg_status tg_gated_attention_train_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                          const float *s, const float *gain, float tau,
+                                          const int32_t *cu_seqlens, int32_t B, int64_t total,
+                                          int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                          tg_bf16 *O, float *lse, float *O32, tg_stream stream);
+
 /* --------------------------------------------------------------------------
  * tg_gated_attention_backward -- gradients of token-gated attention with respect
  * to the key scores, the per-head gains and the temperature: the path by which
@@ -306,6 +316,30 @@ tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16 *Kc, const
                                       int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
                                       float *ds, float *dgain, float *dtau,
                                       void *workspace, size_t workspace_bytes, tg_stream stream);
+
+/* The backward of a packed ragged batch (the training side of
+ * tg_gated_attention_varlen, e.g. a batch of requests each trained under its own
+ * budget).  Request b owns packed rows [cu_seqlens[b], cu_seqlens[b+1]) of Q, Kc, V, s,
+ * O, O32, dO and lse (cu_seqlens: device int32 [B+1], non-decreasing within [0, total])
+ * and attends causally within itself only, so
+ *     ds[j]    = the formula above within j's request,
+ *     dgain[h] = sum over every request,   dtau = sum over every request.
+ * Rows outside every request get ds = 0.  max_seqlen is a host upper bound on any
+ * request's length (it sizes the grid).  workspace: at least
+ * tg_gated_attention_backward_varlen_workspace(total, B, Hq) bytes (each request's rows
+ * padded to whole 128-row blocks), 16-byte aligned, caller-owned.  Malformed cu_seqlens,
+ * or a request longer than max_seqlen, set TG_DEVERR_BAD_SEQLENS and leave the gradients
+ * undefined.  Sizes and the rest as for tg_gated_attention_backward. */
+size_t tg_gated_attention_backward_varlen_workspace(int64_t total, int32_t B, int32_t Hq);
+
+tg_status tg_gated_attention_backward_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                             const float *s, const float *gain, float tau,
+                                             const tg_bf16 *O, const float *O32, const tg_bf16 *dO,
+                                             const float *lse, const int32_t *cu_seqlens, int32_t B,
+                                             int64_t total, int64_t max_seqlen,
+                                             int32_t Hq, int32_t Hkv, int32_t D,
+                                             float *ds, float *dgain, float *dtau,
+                                             void *workspace, size_t workspace_bytes, tg_stream stream);
 
 /* tg_gated_attention_backward_noalloc -- the same backward without a caller
  * workspace and without allocating anything: its scratch is a fixed 4 MiB device

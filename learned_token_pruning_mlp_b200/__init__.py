@@ -22,8 +22,11 @@ from ._lib import (  # noqa: F401
     tg_gated_attention,
     tg_gated_attention_backward,
     tg_gated_attention_backward_noalloc,
+    tg_gated_attention_backward_varlen,
+    tg_gated_attention_backward_varlen_workspace,
     tg_gated_attention_backward_workspace,
     tg_gated_attention_train,
+    tg_gated_attention_train_varlen,
     tg_gated_attention_varlen,
     tg_gather,
     tg_get_device_error,

@@ -60,6 +60,11 @@ _SIGNATURES = {
     "tg_gated_attention_backward_workspace": ([_i64, _i32], ctypes.c_size_t),
     "tg_gated_attention_backward": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp,
                                      _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
+    "tg_gated_attention_train_varlen": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp,
+                                         _vp, _vp, _vp], ctypes.c_int),
+    "tg_gated_attention_backward_varlen_workspace": ([_i64, _i32, _i32], ctypes.c_size_t),
+    "tg_gated_attention_backward_varlen": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64,
+                                            _i32, _i32, _i32, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "tg_gated_attention_backward_noalloc": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i64, _i32, _i32,
                                              _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
     "tg_qkv_rope": ([_vp, _i64, _i32, _vp, _vp, ctypes.c_double, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
@@ -321,6 +326,57 @@ def tg_gated_attention_varlen(Q, Kc, V, s, gain, tau: float, cu_seqlens, max_seq
         _dev(gain, torch.float32, "gain"), float(tau), _dev(cu_seqlens, torch.int32, "cu_seqlens"), B, total,
         int(max_seqlen), Hq, Hkv, D, _dev(O, bf, "O"), _stream(stream)))
     return O
+
+
+def tg_gated_attention_train_varlen(Q, Kc, V, s, gain, tau: float, cu_seqlens, max_seqlen: int, O=None, lse=None,
+                                   O32=None, keep_fp32=True, stream=None):
+    """Training forward of a packed ragged batch: returns (O bf16, lse fp32 [total, Hq], O32 or None)."""
+    total, Hq, D = Q.shape
+    Hkv = Kc.shape[1]
+    B = cu_seqlens.numel() - 1
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty((total, Hq), dtype=torch.float32, device=Q.device)
+    if O32 is None and keep_fp32:
+        O32 = torch.empty((total, Hq, D), dtype=torch.float32, device=Q.device)
+    bf = torch.bfloat16
+    _check("tg_gated_attention_train_varlen", lib().tg_gated_attention_train_varlen(
+        _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _dev(s, torch.float32, "s"),
+        _dev(gain, torch.float32, "gain"), float(tau), _dev(cu_seqlens, torch.int32, "cu_seqlens"), B, total,
+        int(max_seqlen), Hq, Hkv, D, _dev(O, bf, "O"), _dev(lse, torch.float32, "lse"),
+        _dev(O32, torch.float32, "O32"), _stream(stream)))
+    return O, lse, O32
+
+
+def tg_gated_attention_backward_varlen_workspace(total: int, B: int, Hq: int) -> int:
+    return int(lib().tg_gated_attention_backward_varlen_workspace(int(total), int(B), int(Hq)))
+
+
+def tg_gated_attention_backward_varlen(Q, Kc, V, s, gain, tau: float, O, dO, lse, cu_seqlens, max_seqlen: int,
+                                       O32=None, ds=None, dgain=None, dtau=None, workspace=None, stream=None):
+    total, Hq, D = Q.shape
+    Hkv = Kc.shape[1]
+    B = cu_seqlens.numel() - 1
+    dev = gain.device
+    if ds is None:
+        ds = torch.empty(total, dtype=torch.float32, device=dev)
+    if dgain is None:
+        dgain = torch.empty(Hq, dtype=torch.float32, device=dev)
+    if dtau is None:
+        dtau = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = tg_gated_attention_backward_varlen_workspace(total, B, Hq)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    bf = torch.bfloat16
+    _check("tg_gated_attention_backward_varlen", lib().tg_gated_attention_backward_varlen(
+        _dev(Q, bf, "Q"), _dev(Kc, bf, "Kc"), _dev(V, bf, "V"), _dev(s, torch.float32, "s"),
+        _dev(gain, torch.float32, "gain"), float(tau), _dev(O, bf, "O"), _dev(O32, torch.float32, "O32"),
+        _dev(dO, bf, "dO"), _dev(lse, torch.float32, "lse"), _dev(cu_seqlens, torch.int32, "cu_seqlens"), B, total,
+        int(max_seqlen), Hq, Hkv, D, _dev(ds, torch.float32, "ds"), _dev(dgain, torch.float32, "dgain"),
+        _dev(dtau, torch.float32, "dtau"), _dev(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream)))
+    return ds, dgain, dtau
 
 
 def tg_gated_attention_backward_noalloc(Q, Kc, V, s, gain, tau: float, O, dO, lse, O32=None, ds=None, dgain=None,

@@ -650,3 +650,23 @@ extern "C" tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *
   return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, nullptr, nullptr, cs, err)
                   : launch<64>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, nullptr, nullptr, cs, err);
 }
+
+extern "C" tg_status tg_gated_attention_train_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                                     const float *s, const float *gain, float tau,
+                                                     const int32_t *cu_seqlens, int32_t B, int64_t total,
+                                                     int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                                     tg_bf16 *O, float *lse, float *O32, tg_stream stream) {
+  TG_API_ENTRY();
+  if (B < 0) return tg::fail(TG_ERR_INVALID_ARG, "B must be >= 0");
+  if (max_seqlen < 0 || max_seqlen > total) return tg::fail(TG_ERR_INVALID_ARG, "max_seqlen must be in [0, total]");
+  if (B > 0 && !cu_seqlens) return tg::fail(TG_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  tg_status st = validate(Q, Kc, V, s, gain, tau, total, Hq, Hkv, D, O);
+  if (st != TG_OK || total == 0 || B == 0) return st;
+  if (!lse) return tg::fail(TG_ERR_INVALID_ARG, "lse is NULL");
+  if (O32 && !tg::aligned16(O32)) return tg::fail(TG_ERR_ALIGNMENT, "O32 must be 16-byte aligned");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch<128>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, lse, O32, cs, err)
+                  : launch<64>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, lse, O32, cs, err);
+}

@@ -30,6 +30,10 @@
 //   3. reduce: ds, dgain and dtau from the per-(head, key) column sums and the
 //      per-CTA temperature partials, each summed in a fixed order, so the result is
 //      deterministic.
+// Packed ragged batches (cu_seqlens): each request attends within itself only, so its
+// rows get their own span of every per-head workspace vector, padded to whole 128-row
+// blocks; a CTA works on (key block, request, head) and the reduction maps packed rows
+// back to their request's span.  dgain and dtau sum over every request.
 #include <algorithm>
 #include <cmath>
 
@@ -68,45 +72,96 @@ struct BwdCtl {
   float tau_part[8];
 };
 
-// Workspace (fp32): -lse2 [Hq][S_pad], -Delta [Hq][S_pad], colsum [Hq][S_pad], tau partials [Hq][n_kb].
+// Workspace (fp32), ``stride`` rows per head (a multiple of 128): -lse2 [Hq][stride],
+// -Delta [Hq][stride], colsum [Hq][stride], tau partials [Hq][stride / 128].
 struct Workspace {
   float *nlse2, *ndelta, *colsum, *taup;
+  int64_t stride;
 };
 
 __host__ __device__ inline int64_t padded_rows(int64_t S) { return (S + kBK - 1) / kBK * kBK; }
 
-inline size_t workspace_bytes(int64_t S, int32_t Hq) {
-  const int64_t sp = padded_rows(S);
-  const size_t floats = static_cast<size_t>(Hq) * (3 * static_cast<size_t>(sp) + static_cast<size_t>(sp / kBK));
+// Workspace rows per head: one sequence of S rows, or a packed batch of ``total`` rows in
+// B requests (each request padded to whole blocks: at most total + 127 B rows).
+inline int64_t ws_stride(int64_t total, int32_t B) { return B <= 1 ? padded_rows(total) : padded_rows(total) + kBK * B; }
+
+inline size_t workspace_bytes_stride(int64_t stride, int32_t Hq) {
+  const size_t floats = static_cast<size_t>(Hq) * (3 * static_cast<size_t>(stride) + static_cast<size_t>(stride / kBK));
   return (floats * 4 + 255) / 256 * 256;
 }
 
-inline Workspace carve(void *base, int64_t S, int32_t Hq) {
-  const size_t sp = static_cast<size_t>(padded_rows(S));
+inline size_t workspace_bytes(int64_t S, int32_t Hq) { return workspace_bytes_stride(padded_rows(S), Hq); }
+
+inline Workspace carve(void *base, int64_t stride, int32_t Hq) {
+  const size_t sp = static_cast<size_t>(stride);
   float *f = static_cast<float *>(base);
-  return Workspace{f, f + Hq * sp, f + 2 * Hq * sp, f + 3 * Hq * sp};
+  return Workspace{f, f + Hq * sp, f + 2 * Hq * sp, f + 3 * Hq * sp, stride};
+}
+
+// The requests of a packed batch.  Request b owns packed rows [s0, s0 + len) of Q, K, V,
+// dO, O, lse and s, and rows [p0, p0 + padded_rows(len)) of every per-head workspace
+// vector.  Without cu_seqlens there is one request of ``total`` rows at p0 = 0.
+struct Segs {
+  const int32_t *cu;  // device int32 [B + 1], or nullptr
+  int B;
+  int64_t total;
+  int64_t max_len;    // host bound on a request's length (it sizes the grids)
+};
+struct Seg {
+  int64_t s0, len, p0;
+  bool valid;  // cu_seqlens non-decreasing within [0, total] up to this request, length <= max_len
+};
+
+__device__ inline Seg seg_of(const Segs &sg, int64_t stride, int b) {
+  Seg r{0, sg.total, 0, true};
+  if (!sg.cu) return r;
+  int64_t prev = sg.cu[0], p = 0;
+  bool ok = prev >= 0 && prev <= sg.total;
+  for (int i = 0; i < b && ok; ++i) {
+    const int64_t nx = sg.cu[i + 1];
+    ok = nx >= prev && nx <= sg.total;
+    p += padded_rows(nx - prev);
+    prev = nx;
+  }
+  const int64_t e = ok ? static_cast<int64_t>(sg.cu[b + 1]) : prev;
+  ok = ok && e >= prev && e <= sg.total && e - prev <= sg.max_len && p + padded_rows(e - prev) <= stride;
+  r.s0 = prev;
+  r.len = ok ? e - prev : 0;
+  r.p0 = p;
+  r.valid = ok;
+  return r;
 }
 
 // ------------------------------------------------------------------------------ prep
 // One warp per (row, head) of the padded range, the whole range in one grid: Delta =
 // dO . O (fp32), from the fp32 output with one 16-byte load per lane (D = 128) when it
 // is given, and the lse converted to base 2; both stored negated, per head.
+// Warps cover (request, padded row of the request, head); rows past a request's length
+// are its padding.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16 *__restrict__ O,
                                                             const float *__restrict__ O32,
                                                             const __nv_bfloat16 *__restrict__ dO,
-                                                            const float *__restrict__ lse, int64_t S, int64_t S_pad,
-                                                            int Hq, Workspace ws) {
+                                                            const float *__restrict__ lse, Segs sg, int64_t Lpad,
+                                                            int Hq, Workspace ws, uint32_t *err) {
   tg::pdl_wait();
   tg::pdl_trigger();
   constexpr int kPer = D / 32;  // elements per lane (2 or 4)
   const int lane = threadIdx.x & 31;
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (w >= S_pad * Hq) return;  // whole warps
-  const int64_t i = w / Hq;
+  if (w >= static_cast<int64_t>(sg.B) * Lpad * Hq) return;  // whole warps
   const int h = static_cast<int>(w % Hq);
+  const int64_t lr = (w / Hq) % Lpad;
+  const int b = static_cast<int>(w / Hq / Lpad);
+  const Seg sgm = seg_of(sg, ws.stride, b);
+  if (!sgm.valid) {
+    if (lane == 0 && lr == 0 && h == 0) tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
+    return;
+  }
+  if (lr >= padded_rows(sgm.len)) return;
+  const int64_t i = sgm.s0 + lr;  // packed row (a real one when lr < len)
   float nd = 0.f, nl = -INFINITY;
-  if (i < S) {
+  if (lr < sgm.len) {
     const int64_t off = (i * Hq + h) * D + lane * kPer;
     float o[kPer], d[kPer];
     if constexpr (kPer == 4) {
@@ -151,8 +206,8 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16 
     nl = -lse[i * Hq + h] * kLog2e;
   }
   if (lane == 0) {
-    ws.ndelta[h * S_pad + i] = nd;
-    ws.nlse2[h * S_pad + i] = nl;
+    ws.ndelta[h * ws.stride + sgm.p0 + lr] = nd;
+    ws.nlse2[h * ws.stride + sgm.p0 + lr] = nl;
   }
 }
 
@@ -161,8 +216,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const float *__restrict__ key_scores, const float *__restrict__ gain, float c_log2, int64_t S,
-                    int64_t S_pad, int Hq, int Hkv, Workspace ws, uint32_t *err) {
+                    const float *__restrict__ key_scores, const float *__restrict__ gain, float c_log2, Segs sg,
+                    int Hq, int Hkv, Workspace ws, uint32_t *err) {
   using C = BwdCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -176,11 +231,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *sCs = sDl + kAux * kBQ;                                     // [kBK] second warpgroup's column sums
   BwdCtl *ctl = reinterpret_cast<BwdCtl *>(sCs + kBK);
 
-  const int n_kb = static_cast<int>(S_pad / kBK);
-  const int kb = static_cast<int>(blockIdx.x) / Hq;  // ascending: the longest key blocks first
+  // (key block, request, head); key blocks ascending: the longest ones first
+  const int per_kb = sg.B * Hq;
+  const int kb = static_cast<int>(blockIdx.x) / per_kb;
+  const int b = (static_cast<int>(blockIdx.x) % per_kb) / Hq;
   const int h = static_cast<int>(blockIdx.x) % Hq;
   const int g = h / (Hq / Hkv);
+  const Seg sgm = seg_of(sg, ws.stride, b);
+  const int n_kb = static_cast<int>(padded_rows(sgm.len) / kBK);
+  if (!sgm.valid || kb >= n_kb) return;              // uniform over the CTA, before any set-up
   const int n_steps = n_kb - kb;                     // query blocks kb .. n_kb-1
+  const int64_t s0 = sgm.s0;
+  const int64_t wrow0 = h * ws.stride + sgm.p0;      // the request's span of this head's vectors
   const int warp = tg::warp_id();
   const int lane = threadIdx.x & 31;
 
@@ -228,11 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t kvb = tg::smem_addr(&ctl->kv_full);
     tg::mbar_arrive_expect_tx(kvb, 2 * C::kTileBytes);
     for (int hf = 0; hf < C::kHalves; ++hf) {
-      tg::tma_load_3d(tg::smem_addr(sK + hf * kHalfBytes), &tm_k, kvb, hf * 64, g, kb * kBK);
-      tg::tma_load_3d(tg::smem_addr(sV + hf * kHalfBytes), &tm_v, kvb, hf * 64, g, kb * kBK);
+      tg::tma_load_3d(tg::smem_addr(sK + hf * kHalfBytes), &tm_k, kvb, hf * 64, g,
+                      static_cast<int32_t>(s0 + kb * kBK));
+      tg::tma_load_3d(tg::smem_addr(sV + hf * kHalfBytes), &tm_v, kvb, hf * 64, g,
+                      static_cast<int32_t>(s0 + kb * kBK));
     }
     for (int n = 0; n < n_steps; ++n) {
-      const int qrow = (kb + n) * kBQ;
+      const int qblk = (kb + n) * kBQ;  // request-relative
+      const int32_t qrow = static_cast<int32_t>(s0 + qblk);
       const int s = n % NS;
       if (!tg::mbar_wait(tg::smem_addr(&ctl->q_empty[s]), ((n / NS) & 1) ^ 1, abort_flag)) break;
       const uint32_t qf = tg::smem_addr(&ctl->q_full[s]);
@@ -245,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tg::mbar_wait(tg::smem_addr(&ctl->aux_empty[a]), ((n / kAux) & 1) ^ 1, abort_flag)) break;
       const uint32_t af = tg::smem_addr(&ctl->aux_full[a]);
       tg::mbar_arrive_expect_tx(af, 2 * kBQ * 4);
-      tg::bulk_load(tg::smem_addr(sL + a * kBQ), ws.nlse2 + h * S_pad + qrow, kBQ * 4, af);
-      tg::bulk_load(tg::smem_addr(sDl + a * kBQ), ws.ndelta + h * S_pad + qrow, kBQ * 4, af);
+      tg::bulk_load(tg::smem_addr(sL + a * kBQ), ws.nlse2 + wrow0 + qblk, kBQ * 4, af);
+      tg::bulk_load(tg::smem_addr(sDl + a * kBQ), ws.ndelta + wrow0 + qblk, kBQ * 4, af);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -296,8 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - 4) >> 2;       // query columns 64*grp .. 64*grp+63
     const int quarter = warp & 3;          // TMEM lane quarter
     const int r = quarter * 32 + lane;     // key within the block
-    const int64_t j = static_cast<int64_t>(kb) * kBK + r;
-    const float bj = j < S ? gain[h] * kLog2e * key_scores[j] : -INFINITY;
+    const int64_t j = static_cast<int64_t>(kb) * kBK + r;  // request-relative key
+    const float bj = j < sgm.len ? gain[h] * kLog2e * key_scores[s0 + j] : -INFINITY;
     const uint64_t bj2 = tg::f2_pack(bj, bj);
     const uint64_t c2 = tg::f2_pack(c_log2, c_log2);
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -351,12 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) ctl->tau_part[warp - 4] = tacc;
     asm volatile("bar.sync 1, 256;" ::: "memory");  // the two warpgroups
     if (grp == 0) {
-      ws.colsum[h * S_pad + j] = colsum + sCs[r];
+      ws.colsum[wrow0 + j] = colsum + sCs[r];
       if (r == 0) {
         float t = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) t += ctl->tau_part[w];
-        ws.taup[h * n_kb + kb] = t;
+        ws.taup[h * (ws.stride / kBK) + sgm.p0 / kBK + kb] = t;
       }
     }
   }
@@ -371,34 +436,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ reduce
-// Blocks [0, nb_ds): ds for 256 keys each; blocks nb_ds + h: dgain[h]; the last block:
-// dtau.  Every sum runs in a fixed order.
+// Blocks [0, nb_ds): ds for 256 packed keys each; blocks nb_ds + h: dgain[h]; the last
+// block: dtau.  Every sum runs in a fixed order (requests in order), so the result is
+// deterministic.  Rows outside every request (a batch that does not cover [0, total))
+// get ds = 0; a malformed batch leaves the outputs undefined (flagged by the prep).
 __global__ void __launch_bounds__(256) attn_bwd_reduce_kernel(Workspace ws, const float *__restrict__ key_scores,
-                                                              const float *__restrict__ gain, int64_t S,
-                                                              int64_t S_pad, int Hq, int nb_ds, float inv_sqrt_d,
-                                                              float *__restrict__ ds, float *__restrict__ dgain,
-                                                              float *__restrict__ dtau) {
+                                                              const float *__restrict__ gain, Segs sg, int Hq,
+                                                              int nb_ds, float inv_sqrt_d, float *__restrict__ ds,
+                                                              float *__restrict__ dgain, float *__restrict__ dtau) {
   tg::pdl_wait();
   tg::pdl_trigger();
   __shared__ float red[256];
-  const int b = static_cast<int>(blockIdx.x);
+  const int blk = static_cast<int>(blockIdx.x);
   const int t = threadIdx.x;
-  if (b < nb_ds) {
-    const int64_t j = static_cast<int64_t>(b) * 256 + t;
-    if (j < S) {
+  if (blk < nb_ds) {
+    const int64_t j = static_cast<int64_t>(blk) * 256 + t;
+    if (j < sg.total) {
       float acc = 0.f;
-      for (int h = 0; h < Hq; ++h) acc = fmaf(gain[h], ws.colsum[h * S_pad + j], acc);
+      for (int b = 0; b < sg.B; ++b) {  // the request that holds packed row j
+        const Seg sgm = seg_of(sg, ws.stride, b);
+        if (!sgm.valid) break;
+        if (j >= sgm.s0 && j < sgm.s0 + sgm.len) {
+          const int64_t wr = sgm.p0 + (j - sgm.s0);
+          for (int h = 0; h < Hq; ++h) acc = fmaf(gain[h], ws.colsum[h * ws.stride + wr], acc);
+          break;
+        }
+      }
       ds[j] = acc;
     }
     return;
   }
-  const int h = b - nb_ds;  // h == Hq: the temperature
+  const int h = blk - nb_ds;  // h == Hq: the temperature
   float acc = 0.f;
-  if (h < Hq) {
-    for (int64_t j = t; j < S; j += 256) acc = fmaf(key_scores[j], ws.colsum[h * S_pad + j], acc);
-  } else {
-    const int64_t n = static_cast<int64_t>(Hq) * (S_pad / kBK);
-    for (int64_t i = t; i < n; i += 256) acc += ws.taup[i];
+  for (int b = 0; b < sg.B; ++b) {
+    const Seg sgm = seg_of(sg, ws.stride, b);
+    if (!sgm.valid) break;
+    if (h < Hq) {
+      const float *cs = ws.colsum + h * ws.stride + sgm.p0;
+      for (int64_t jl = t; jl < sgm.len; jl += 256) acc = fmaf(key_scores[sgm.s0 + jl], cs[jl], acc);
+    } else {
+      const int64_t nkb = padded_rows(sgm.len) / kBK;
+      for (int64_t i = t; i < nkb * Hq; i += 256)
+        acc += ws.taup[(i / nkb) * (ws.stride / kBK) + sgm.p0 / kBK + (i % nkb)];
+    }
   }
   red[t] = acc;
   __syncthreads();
@@ -423,11 +503,13 @@ bool tmap3(CUtensorMap *m, const void *base, int D, int heads, int64_t rows) {
 
 template <int D>
 tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain,
-                     float tau, const tg_bf16 *O, const float *O32, const tg_bf16 *dO, const float *lse, int64_t S,
-                     int32_t Hq, int32_t Hkv, const Workspace &ws, cudaStream_t stream, uint32_t *err) {
+                     float tau, const tg_bf16 *O, const float *O32, const tg_bf16 *dO, const float *lse,
+                     const Segs &sg, int32_t Hq, int32_t Hkv, const Workspace &ws, cudaStream_t stream,
+                     uint32_t *err) {
   using C = BwdCfg<D>;
-  const int64_t S_pad = padded_rows(S);
-  const int n_kb = static_cast<int>(S_pad / kBK);
+  const int64_t S = sg.total;
+  const int64_t Lpad = padded_rows(sg.max_len);
+  const int n_kb = static_cast<int>(Lpad / kBK);
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
   if (!tmap3(&tm_q, Q, D, Hq, S) || !tmap3(&tm_k, Kc, D, Hkv, S) || !tmap3(&tm_v, V, D, Hkv, S) ||
       !tmap3(&tm_do, dO, D, Hq, S))
@@ -447,15 +529,17 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
     return TG_OK;
   });
   if (setup != TG_OK) return setup;
-  const int64_t prep_warps = S_pad * Hq;  // below 2^31 (checked by the caller)
+  const int64_t prep_warps = static_cast<int64_t>(sg.B) * Lpad * Hq;  // checked by the caller
   const unsigned prep_grid = static_cast<unsigned>((prep_warps + 7) / 8);
   cudaError_t e = tg::launch_pdl(attn_bwd_prep_kernel<D>, dim3(prep_grid), dim3(256), 0, stream,
                                  reinterpret_cast<const __nv_bfloat16 *>(O), O32,
-                                 reinterpret_cast<const __nv_bfloat16 *>(dO), lse, S, S_pad, static_cast<int>(Hq), ws);
+                                 reinterpret_cast<const __nv_bfloat16 *>(dO), lse, sg, Lpad, static_cast<int>(Hq), ws,
+                                 err);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "attn_bwd_prep_kernel launch: %s", cudaGetErrorString(e));
   const float c_log2 = tau / std::sqrt(static_cast<float>(D)) * kLog2e;
-  e = tg::launch_pdl(attn_bwd_kernel<D>, dim3(static_cast<unsigned>(n_kb * Hq)), dim3(kThreads), C::kSmem, stream, tm_q,
-                     tm_k, tm_v, tm_do, s, gain, c_log2, S, S_pad, static_cast<int>(Hq), static_cast<int>(Hkv), ws, err);
+  const int64_t grid = static_cast<int64_t>(n_kb) * sg.B * Hq;
+  e = tg::launch_pdl(attn_bwd_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::kSmem, stream, tm_q,
+                     tm_k, tm_v, tm_do, s, gain, c_log2, sg, static_cast<int>(Hq), static_cast<int>(Hkv), ws, err);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "attn_bwd_kernel launch: %s", cudaGetErrorString(e));
   return TG_OK;
 }
@@ -466,15 +550,55 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
 
-tg_status launch_reduce(const Workspace &ws, const float *s, const float *gain, int64_t S, int32_t Hq, int32_t D,
+tg_status launch_reduce(const Workspace &ws, const float *s, const float *gain, const Segs &sg, int32_t Hq, int32_t D,
                         float *ds, float *dgain, float *dtau, cudaStream_t stream) {
-  const int nb_ds = static_cast<int>((S + 255) / 256);
+  const int nb_ds = static_cast<int>((sg.total + 255) / 256);
   const cudaError_t e =
       tg::launch_pdl(attn_bwd_reduce_kernel, dim3(static_cast<unsigned>(nb_ds + Hq + 1)), dim3(256), 0, stream, ws, s,
-                     gain, S, padded_rows(S), static_cast<int>(Hq), nb_ds, 1.0f / std::sqrt(static_cast<float>(D)), ds,
-                     dgain, dtau);
+                     gain, sg, static_cast<int>(Hq), nb_ds, 1.0f / std::sqrt(static_cast<float>(D)), ds, dgain, dtau);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "attn_bwd_reduce_kernel launch: %s", cudaGetErrorString(e));
   return TG_OK;
+}
+
+// The backward of one sequence (cu_seqlens = nullptr, B = 1) or of a packed batch.
+tg_status backward_impl(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain,
+                        float tau, const tg_bf16 *O, const float *O32, const tg_bf16 *dO, const float *lse,
+                        const int32_t *cu_seqlens, int32_t B, int64_t S, int64_t max_len, int32_t Hq, int32_t Hkv,
+                        int32_t D, float *ds, float *dgain, float *dtau, void *workspace, size_t workspace_size,
+                        tg_stream stream) {
+  if (S < 0) return tg::fail(TG_ERR_INVALID_ARG, "S must be >= 0");
+  if (B < 1) return tg::fail(TG_ERR_INVALID_ARG, "B must be >= 1");
+  if (max_len < 0 || max_len > S) return tg::fail(TG_ERR_INVALID_ARG, "max_seqlen must be in [0, total]");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return tg::fail(TG_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv");
+  if (D != 64 && D != 128) return tg::fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+  if (!std::isfinite(tau)) return tg::fail(TG_ERR_INVALID_ARG, "tau must be finite");
+  const int64_t stride = cu_seqlens ? ws_stride(S, B) : padded_rows(S);
+  if (stride * Hq > (int64_t(1) << 31) - 1 || padded_rows(max_len) * B * Hq > (int64_t(1) << 31) - 1)
+    return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
+  if (!gain || !dgain || !dtau) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (S > 0 && (!Q || !Kc || !V || !s || (!O && !O32) || !dO || !lse || !ds || !workspace))
+    return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
+  const size_t need = workspace_bytes_stride(stride, Hq);
+  if (S > 0 && workspace_size < need)
+    return tg::fail(TG_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu bytes needed", workspace_size, need);
+  if (S > 0 && (!tg::aligned16(Q) || !tg::aligned16(Kc) || !tg::aligned16(V) || !tg::aligned16(dO) ||
+                !tg::aligned16(O) || !tg::aligned16(O32) || !tg::aligned16(workspace)))
+    return tg::fail(TG_ERR_ALIGNMENT, "Q, Kc, V, O, O32, dO and workspace must be 16-byte aligned");
+  uint32_t *err = tg::device_error_word();
+  if (!err) return TG_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Segs sg{cu_seqlens, cu_seqlens ? B : 1, S, cu_seqlens ? max_len : S};
+  const Workspace ws = S > 0 ? carve(workspace, stride, Hq) : Workspace{nullptr, nullptr, nullptr, nullptr, stride};
+  if (S > 0 && max_len > 0) {
+    const tg_status r = D == 64 ? launch_bwd<64>(Q, Kc, V, s, gain, tau, O, O32, dO, lse, sg, Hq, Hkv, ws, st, err)
+                                : launch_bwd<128>(Q, Kc, V, s, gain, tau, O, O32, dO, lse, sg, Hq, Hkv, ws, st, err);
+    if (r != TG_OK) return r;
+  }
+  // with no work the reduction still writes the (zero) gradients: its loops find no rows
+  const Segs sg_reduce = (S > 0 && max_len > 0) ? sg : Segs{nullptr, 0, S, 0};
+  const tg_status r = launch_reduce(ws, s, gain, sg_reduce, Hq, D, ds, dgain, dtau, st);
+  if (r != TG_OK) return r;
+  return tg::check_launch("tg_gated_attention_backward");
 }
 
 }  // namespace
@@ -484,6 +608,11 @@ extern "C" size_t tg_gated_attention_backward_workspace(int64_t S, int32_t Hq) {
   return workspace_bytes(S, Hq);
 }
 
+extern "C" size_t tg_gated_attention_backward_varlen_workspace(int64_t total, int32_t B, int32_t Hq) {
+  if (total < 0 || B < 1 || Hq <= 0) return 0;
+  return workspace_bytes_stride(ws_stride(total, B), Hq);
+}
+
 extern "C" tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
                                                  const float *s, const float *gain, float tau, const tg_bf16 *O,
                                                  const float *O32, const tg_bf16 *dO, const float *lse, int64_t S,
@@ -491,32 +620,22 @@ extern "C" tg_status tg_gated_attention_backward(const tg_bf16 *Q, const tg_bf16
                                                  int32_t Hkv, int32_t D, float *ds, float *dgain, float *dtau,
                                                  void *workspace, size_t workspace_size, tg_stream stream) {
   TG_API_ENTRY();
-  if (S < 0) return tg::fail(TG_ERR_INVALID_ARG, "S must be >= 0");
-  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return tg::fail(TG_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv");
-  if (D != 64 && D != 128) return tg::fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
-  if (!std::isfinite(tau)) return tg::fail(TG_ERR_INVALID_ARG, "tau must be finite");
-  if (padded_rows(S) * Hq > (int64_t(1) << 31) - 1) return tg::fail(TG_ERR_UNSUPPORTED, "S * Hq must be below 2^31");
-  if (!gain || !dgain || !dtau) return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
-  if (S > 0 && (!Q || !Kc || !V || !s || (!O && !O32) || !dO || !lse || !ds || !workspace))
-    return tg::fail(TG_ERR_INVALID_ARG, "null pointer");
-  const size_t need = workspace_bytes(S, Hq);
-  if (S > 0 && workspace_size < need)
-    return tg::fail(TG_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu bytes needed", workspace_size, need);
-  if (S > 0 && (!tg::aligned16(Q) || !tg::aligned16(Kc) || !tg::aligned16(V) || !tg::aligned16(dO) ||
-                !tg::aligned16(O) || !tg::aligned16(O32) || !tg::aligned16(workspace)))
-    return tg::fail(TG_ERR_ALIGNMENT, "Q, Kc, V, O, O32, dO and workspace must be 16-byte aligned");
-  uint32_t *err = tg::device_error_word();
-  if (!err) return TG_ERR_CUDA;
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Workspace ws = S > 0 ? carve(workspace, S, Hq) : Workspace{nullptr, nullptr, nullptr, nullptr};
-  if (S > 0) {
-    const tg_status r = D == 64 ? launch_bwd<64>(Q, Kc, V, s, gain, tau, O, O32, dO, lse, S, Hq, Hkv, ws, st, err)
-                                : launch_bwd<128>(Q, Kc, V, s, gain, tau, O, O32, dO, lse, S, Hq, Hkv, ws, st, err);
-    if (r != TG_OK) return r;
-  }
-  const tg_status r = launch_reduce(ws, s, gain, S, Hq, D, ds, dgain, dtau, st);
-  if (r != TG_OK) return r;
-  return tg::check_launch("tg_gated_attention_backward");
+  return backward_impl(Q, Kc, V, s, gain, tau, O, O32, dO, lse, nullptr, 1, S, S, Hq, Hkv, D, ds, dgain, dtau,
+                       workspace, workspace_size, stream);
+}
+
+extern "C" tg_status tg_gated_attention_backward_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
+                                                        const float *s, const float *gain, float tau, const tg_bf16 *O,
+                                                        const float *O32, const tg_bf16 *dO, const float *lse,
+                                                        const int32_t *cu_seqlens, int32_t B, int64_t total,
+                                                        int64_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                                        float *ds, float *dgain, float *dtau, void *workspace,
+                                                        size_t workspace_size, tg_stream stream) {
+  TG_API_ENTRY();
+  if (B < 1) return tg::fail(TG_ERR_INVALID_ARG, "B must be >= 1");
+  if (!cu_seqlens) return tg::fail(TG_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  return backward_impl(Q, Kc, V, s, gain, tau, O, O32, dO, lse, cu_seqlens, B, total, max_seqlen, Hq, Hkv, D, ds,
+                       dgain, dtau, workspace, workspace_size, stream);
 }
 
 extern "C" tg_status tg_gated_attention_backward_noalloc(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,

@@ -56,6 +56,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep until the phase completes
+// (or about ``hint_ns`` passes) instead of spinning, so a waiting warp leaves its
+// sub-partition's issue slots to the warps that work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspend hint of the waits below: long against any hand-off (the hardware resumes the
+// thread when the phase completes), short against the wait limit.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
 // Wait until the phase with the given parity of the mbarrier has completed.
 // Returns false (and raises *abort) when the wait limit passes or when another
 // thread of the CTA has already raised *abort.
@@ -63,15 +82,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        return false;
-      }
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      return false;
     }
   }
 }

@@ -147,6 +147,27 @@ def test_backward_workspace_size_and_argument_checks(L):
     assert L.tg_gated_attention_train(p, p, p, p, p, f, 10, 4, 2, 64, p, p, ctypes.c_void_p(4104), None) == 3
 
 
+def test_backward_varlen_workspace_and_argument_checks(L):
+    L.tg_gated_attention_backward_varlen_workspace.restype = ctypes.c_size_t
+    # 1000 packed rows in 3 requests: 1024 + 3 * 128 = 1408 rows per head (each request padded)
+    assert L.tg_gated_attention_backward_varlen_workspace(1000, 3, 16) == (4 * 16 * (3 * 1408 + 11) + 255) // 256 * 256
+    assert L.tg_gated_attention_backward_varlen_workspace(1000, 0, 16) == 0
+    assert L.tg_gated_attention_backward_varlen_workspace(-1, 2, 16) == 0
+    p = ctypes.c_void_p(4096)
+    f = ctypes.c_float(1.0)
+    big = ctypes.c_size_t(1 << 30)
+    args = lambda cu, B, total, mx, n=big: (p, p, p, p, p, f, p, None, p, p, cu, B, total, mx, 4, 2, 64, p, p, p,  # noqa: E731
+                                            p, n, None)
+    assert L.tg_gated_attention_backward_varlen(*args(p, 0, 100, 50)) == 1        # B < 1
+    assert L.tg_gated_attention_backward_varlen(*args(None, 2, 100, 50)) == 1     # cu_seqlens NULL
+    assert L.tg_gated_attention_backward_varlen(*args(p, 2, 100, 101)) == 1       # max_seqlen > total
+    assert L.tg_gated_attention_backward_varlen(*args(p, 2, 100, 50, n=ctypes.c_size_t(4 * 4 * 3 * 256))) == 1
+    assert "workspace" in _detail(L)
+    assert L.tg_gated_attention_train_varlen(p, p, p, p, p, f, None, 2, 10, 5, 4, 2, 64, p, p, None, None) == 1
+    assert L.tg_gated_attention_train_varlen(p, p, p, p, p, f, p, 2, 10, 11, 4, 2, 64, p, p, None, None) == 1
+    assert L.tg_gated_attention_train_varlen(p, p, p, p, p, f, p, 2, 10, 5, 4, 2, 64, p, None, None, None) == 1
+
+
 def test_backward_noalloc_rejects_sizes_beyond_its_static_scratch(L):
     p = ctypes.c_void_p(4096)
     f = ctypes.c_float(1.0)
