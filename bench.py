@@ -322,6 +322,28 @@ def run_tokengate(args, world, rank, local):
         torch.cuda.synchronize()
         return max_over_ranks(s0.elapsed_time(s1) / sel_iters * 1e3, world)
 
+    # The select path's marginal cost inside the step: the same steps with the 27
+    # attention layers alone, timed the same way; the difference is what gate -> top-K
+    # -> gather add to a step once their launches overlap their neighbours' (the
+    # event-bracketed in-step figure above cuts that overlap at both ends).
+    def attention_only():
+        for l in range(L):
+            Q, Kc, V = layers[l]
+            tg.tg_gated_attention(Q, Kc, V, s_k, dv["gain"], tau, O=outs[l])
+
+    for _ in range(3):
+        attention_only()
+    barrier(world)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        attention_only()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    attn_only_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, world)
+    marginal_us = (ms_per_step - attn_only_ms) * 1e3
+
     sel_b2b_us = time_select(False)
     sel_b2b_gbs = sel_bytes / (sel_b2b_us * 1e-6) / 1e9
     own_us = time_select(True)
@@ -376,6 +398,14 @@ def run_tokengate(args, world, rank, local):
                         "in_step_us": round(sel_mean * 1e3, 2),
                         "in_step_gbs": round(sel_gbs, 1),
                         "in_step_frac_of_hbm": round(sel_gbs / peaks["hbm_gbs"], 4),
+                        "in_step_timing": "CUDA events around gate -> top-K -> gather in every timed step (the "
+                                          "events stop the launches overlapping the neighbouring kernels)",
+                        "in_step_marginal_us": round(marginal_us, 2),
+                        "in_step_marginal_timing": f"step time minus the same {args.steps} steps of the "
+                                                   f"{L} attention layers alone ({attn_only_ms:.4f} ms per step): "
+                                                   f"what the select path adds to a step once its kernels "
+                                                   f"overlap the compute-bound attention's first and last "
+                                                   f"waves (not a bandwidth figure)",
                         "gate_scores_chain": {
                             "us": round(own_us, 2), "gbs": round(own_gbs, 1),
                             "frac_of_hbm": round(own_gbs / peaks["hbm_gbs"], 4),

@@ -11,13 +11,16 @@
 // threads each; every thread owns 16 consecutive positions (loaded with 16-byte
 // vector loads) and keeps their 32-bit order keys in registers (131072 positions per
 // cluster; longer requests re-derive the keys from the scores on every pass).  Up to
-// four 8-bit radix passes find the K-th largest key: each CTA builds a shared-memory
-// histogram of the remaining candidates, one cluster barrier publishes it, 256
-// threads sum the eight CTAs' histograms through distributed shared memory and one
-// warp scans the 256 totals, so every CTA agrees on the digit without touching
-// global memory.  A pass whose chosen bin holds exactly the keys still needed ends
-// the search early.  Histograms alternate between two buffers, so one barrier per
-// pass suffices.  The ordered compaction needs one scan of packed (tie, keep) counts
+// three radix passes over 11-, 11- and 10-bit digits find the K-th largest key (each
+// cluster barrier costs about a microsecond, so fewer, wider passes win: continuous
+// scores resolve after two): each CTA builds a shared-memory histogram of the
+// remaining candidates, one cluster barrier publishes it, the CTA's threads sum the
+// eight CTAs' histograms through distributed shared memory and one warp scans the
+// totals, so every CTA agrees on the digit without touching global memory.  A pass
+// whose chosen bin holds exactly the keys still needed ends the search early.
+// Histograms alternate between two buffers, so one barrier per pass suffices.  When
+// the first digit's histogram comes precomputed (tg_select_fused: the gate's epilogue
+// counts the top 8 bits), the passes use four 8-bit digits instead.  The ordered compaction needs one scan of packed (tie, keep) counts
 // per CTA and one exchange of the per-CTA totals.  No workspace, no global atomics,
 // one launch for a single request.
 #include <cooperative_groups.h>
@@ -38,15 +41,18 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kItems = 16;                        // consecutive positions per thread
 constexpr int kRound = kThreads * kItems;         // positions per CTA per round (16384)
-constexpr int kBins = 256;                        // 8-bit digits, four passes at most
+constexpr int kBins = 2048;                       // up to 11-bit digits
+constexpr int kPassBins8 = 256;                   // the precomputed first digit: 8 bits
+constexpr int kCoarse = 256;                      // coarse bins of the two-level digit search
 
 using tg::order_key;
 
 struct TopkShared {
   uint32_t hist[2][kBins];     // double-buffered per-CTA histograms (read by the cluster)
-  uint32_t tot[kBins];         // cluster totals of the current pass
+  uint32_t coarse[2][kCoarse]; // the same histograms folded to 256 coarse bins (read by the cluster)
+  uint32_t fine[kBins / kCoarse];  // cluster totals of the chosen coarse bin's fine bins
   uint32_t wsum[kWarps + 1];
-  uint32_t sel_digit, sel_above, sel_count;
+  uint32_t sel_digit, sel_above, sel_count, sel_cbin;
   long long exch[2];           // ties (key == T) and certain keeps of this CTA: read by the cluster
   long long bcast[2];          // tie_base, out_base
 };
@@ -79,52 +85,67 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, TopkShared &sh, 
   return res;
 }
 
-// Sum the eight CTAs' histograms of buffer ``buf`` (one bin per thread of the first 256),
-// then let warp 0 find the digit of the remaining-th largest candidate, scanning bins
-// from 255 down.  Publishes sel_digit, sel_above (candidates in higher bins) and
-// sel_count (candidates in the chosen bin); sel_digit = 256 if none qualifies.
-__device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster, TopkShared &sh, int buf,
-                                                     uint32_t remaining) {
-  if (threadIdx.x < kBins) {
+// Fold this CTA's histogram of buffer ``buf`` (nbins bins) into 256 coarse bins, g =
+// nbins / 256 consecutive bins each (a copy when g = 1).  Runs before the cluster
+// barrier that publishes the histograms, so the cluster reads the folded bins.
+__device__ __forceinline__ void fold_coarse(TopkShared &sh, int buf, int nbins) {
+  const int g = nbins / kCoarse;
+  if (threadIdx.x < kCoarse) {
     uint32_t c = 0;
+    for (int j = 0; j < g; ++j) c += sh.hist[buf][threadIdx.x * g + j];
+    sh.coarse[buf][threadIdx.x] = c;
+  }
+}
+
+// Find the digit of the remaining-th largest candidate over the whole cluster, in two
+// levels so that few distributed-shared-memory reads are needed: the 256 coarse totals
+// (8 remote reads by each of 256 threads) locate the coarse bin, then the g fine bins
+// of that coarse bin are summed over the eight CTAs.  Publishes sel_digit, sel_above
+// (candidates in higher bins) and sel_count (candidates in the chosen bin);
+// sel_digit = nbins if none qualifies.  The total lands in wsum[kWarps].
+__device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster, TopkShared &sh, int buf,
+                                                     int nbins, uint32_t remaining) {
+  const int g = nbins / kCoarse;
+  const int t = static_cast<int>(threadIdx.x);
+  const int cb = kCoarse - 1 - t;  // coarse bins from the top, one per thread of the first 256
+  uint32_t cnt = 0;
+  if (t < kCoarse) {
 #pragma unroll
-    for (int r = 0; r < kCluster; ++r) c += cluster.map_shared_rank(&sh.hist[buf][0], r)[threadIdx.x];
-    sh.tot[threadIdx.x] = c;
+    for (int r = 0; r < kCluster; ++r) cnt += cluster.map_shared_rank(&sh.coarse[buf][0], r)[cb];
+  }
+  if (t == 0) sh.sel_digit = nbins;  // ordered before the writes below by the scan's barriers
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(cnt, sh, &total);
+  if (t < kCoarse && remaining > 0 && excl < remaining && remaining <= excl + cnt) {
+    sh.sel_cbin = static_cast<uint32_t>(cb);
+    sh.sel_above = excl;
+    sh.sel_count = cnt;
+    if (g == 1) sh.sel_digit = static_cast<uint32_t>(cb);
   }
   __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    uint32_t c[8];
-    uint32_t sum = 0;
+  if (g == 1 || sh.sel_digit != static_cast<uint32_t>(nbins) || remaining == 0 || remaining > total) return;
+  // the fine bins of the chosen coarse bin: lane group j (8 lanes, one per CTA) sums fine
+  // bin cbin * g + g - 1 - j
+  const uint32_t cbin = sh.sel_cbin;
+  if (t < 8 * g) {
+    const int j = t >> 3, r = t & 7;
+    uint32_t c = cluster.map_shared_rank(&sh.hist[buf][0], r)[cbin * g + g - 1 - j];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      c[e] = sh.tot[kBins - 1 - 8 * lane - e];
-      sum += c[e];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-      if (lane >= off) incl += t;
-    }
-    const uint32_t excl = incl - sum;
-    if (lane == 31) {
-      sh.wsum[kWarps] = incl;  // total candidates
-      sh.sel_digit = kBins;
-    }
-    __syncwarp();
-    if (remaining > 0 && excl < remaining && remaining <= incl) {
-      uint32_t run = excl;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (run + c[e] >= remaining) {
-          sh.sel_digit = kBins - 1 - 8 * lane - e;
-          sh.sel_above = run;
-          sh.sel_count = c[e];
-          break;
-        }
-        run += c[e];
+    for (int off = 4; off > 0; off >>= 1) c += __shfl_down_sync(0xFFFFFFFFu, c, off, 8);
+    if (r == 0) sh.fine[j] = c;
+  }
+  __syncthreads();
+  if (t == 0) {
+    uint32_t run = sh.sel_above;
+    for (int j = 0; j < g; ++j) {
+      const uint32_t c = sh.fine[j];
+      if (run + c >= remaining) {
+        sh.sel_digit = cbin * g + g - 1 - j;
+        sh.sel_above = run;
+        sh.sel_count = c;
+        break;
       }
+      run += c;
     }
   }
   __syncthreads();
@@ -259,31 +280,38 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   auto valid = [&](int round, int e) { return round * kRound + static_cast<int>(threadIdx.x) * kItems + e < m; };
 
   if (kResident) load_keys(0);
-  if (threadIdx.x < 2 * kBins) (&sh.hist[0][0])[threadIdx.x] = 0;
+  for (int i = threadIdx.x; i < 2 * kBins; i += kThreads) (&sh.hist[0][0])[i] = 0;
   __syncthreads();
 
-  // ---- radix passes over 8-bit digits, most significant first.  Pass p histograms the
+  // ---- radix passes, most significant digit first: 11, 11 and 10 bits, or four 8-bit
+  // digits when the first digit's histogram is precomputed.  Pass p histograms the
   // candidates (document keys whose higher digits equal the prefix found so far).
+  const bool digits8 = args.hist_parts != nullptr;
+  const int n_pass = digits8 ? 4 : 3;
   uint32_t prefix = 0, pmask = 0;
   uint32_t remaining = static_cast<uint32_t>(k < 0x7FFFFFFFLL ? k : 0x7FFFFFFFLL);
   long long n_doc = 0;
   int mode = 2;          // 0 = keep no document token, 1 = keep all, 2 = threshold
   uint32_t T = 0u;       // keep key > T, plus the first need_eq keys == T in index order
   long long need_eq = 0;
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < n_pass; ++pass) {
     const int buf = pass & 1;
-    const int shift = 24 - 8 * pass;
+    const int width = digits8 ? 8 : (pass < 2 ? 11 : 10);
+    const int shift = digits8 ? 24 - 8 * pass : (pass == 0 ? 21 : (pass == 1 ? 10 : 0));
+    const int nbins = 1 << width;
+    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
     if (pass >= 2) {
       // this buffer was read by every CTA before the cluster barrier of the previous pass
-      if (threadIdx.x < kBins) sh.hist[buf][threadIdx.x] = 0;
+      for (int i = threadIdx.x; i < nbins; i += kThreads) sh.hist[buf][i] = 0;
       __syncthreads();
     }
-    if (pass == 0 && args.hist_parts) {
+    if (pass == 0 && digits8) {
       // the first digit's histogram was built by the producer of the scores: sum this
       // CTA's share of its partial histograms (the cluster reduction adds the shares)
-      if (threadIdx.x < kBins) {
+      if (threadIdx.x < kPassBins8) {
         uint32_t c = 0;
-        for (int p = rank; p < args.n_parts; p += kCluster) c += __ldg(args.hist_parts + p * kBins + threadIdx.x);
+        for (int p = rank; p < args.n_parts; p += kCluster)
+          c += __ldg(args.hist_parts + p * kPassBins8 + threadIdx.x);
         sh.hist[0][threadIdx.x] = c;
       }
     } else {
@@ -291,12 +319,14 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         if (!kResident) load_keys(rd);
 #pragma unroll
         for (int e = 0; e < kItems; ++e)
-          if (keys[e] != 0u && (keys[e] & pmask) == prefix) atomicAdd(&sh.hist[buf][(keys[e] >> shift) & 0xFFu], 1u);
+          if (keys[e] != 0u && (keys[e] & pmask) == prefix) atomicAdd(&sh.hist[buf][(keys[e] >> shift) & dmask], 1u);
       }
     }
     __syncthreads();
+    fold_coarse(sh, buf, nbins);
+    __syncthreads();
     cluster.sync();
-    cluster_select_digit(cluster, sh, buf, remaining);
+    cluster_select_digit(cluster, sh, buf, nbins, remaining);
     if (pass == 0) {
       n_doc = sh.wsum[kWarps];
       if (k > n_doc && rank == 0 && threadIdx.x == 0) tg::set_device_error(err, TG_DEVERR_K_GT_NDOC);
@@ -306,7 +336,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t d = sh.sel_digit;
     const uint32_t above = sh.sel_above, cnt = sh.sel_count;
     prefix |= d << shift;
-    pmask |= 0xFFu << shift;
+    pmask |= dmask << shift;
     remaining -= above;
     if (cnt == remaining) {
       // every candidate of this bin is kept: threshold just below the bin
@@ -314,7 +344,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       need_eq = 0;
       break;
     }
-    if (pass == 3) {
+    if (pass == n_pass - 1) {
       T = prefix;
       need_eq = remaining;
     }
@@ -394,6 +424,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
     }
   }
+  // the last reads of another CTA's shared memory are done: arrive on the cluster
+  // barrier now and wait for the others only before leaving (a CTA's shared memory must
+  // stay until every reader is through), so the compaction overlaps the barrier
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   __syncthreads();
   const long long tie_base = sh.bcast[0], out_base = sh.bcast[1];
 
@@ -436,7 +470,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     run_gtq += rt & 0xFFFFu;
     if (!kResident) __syncthreads();  // the next round's scan reuses the scan buffer
   }
-  cluster.sync();  // no CTA leaves while another may still read its shared memory
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // every CTA is past its remote reads
 }
 
 // Varlen pre-pass (one CTA): kept count of every request, min(k_b, n_doc_b) + question_b,
