@@ -495,8 +495,23 @@ __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__rest
       tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
     s = s < 0 ? 0 : (s > total ? total : s);
     e = e < s ? s : (e > total ? total : e);
+    // document tokens of the request: 16-byte words over its aligned body (nonzero bytes
+    // counted four at a time), single bytes over the unaligned head and tail
     long long cnt = 0;
-    for (int64_t i = s + threadIdx.x; i < e; i += blockDim.x) cnt += mask[i] != 0;
+    const int64_t a0 = (s + 15) & ~int64_t(15), a1 = e & ~int64_t(15);
+    if (a0 < a1) {
+      const uint4 *w = reinterpret_cast<const uint4 *>(mask + a0);
+      const int64_t nw = (a1 - a0) >> 4;
+      for (int64_t q = threadIdx.x; q < nw; q += blockDim.x) {
+        const uint4 v = __ldg(w + q);
+        cnt += (__popc(__vcmpne4(v.x, 0u)) + __popc(__vcmpne4(v.y, 0u)) + __popc(__vcmpne4(v.z, 0u)) +
+                __popc(__vcmpne4(v.w, 0u))) >> 3;
+      }
+      for (int64_t i = s + threadIdx.x; i < a0; i += blockDim.x) cnt += mask[i] != 0;
+      for (int64_t i = a1 + threadIdx.x; i < e; i += blockDim.x) cnt += mask[i] != 0;
+    } else {
+      for (int64_t i = s + threadIdx.x; i < e; i += blockDim.x) cnt += mask[i] != 0;
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) cnt += __shfl_down_sync(0xFFFFFFFFu, cnt, off);
     if (lane == 0) red[warp] = cnt;
