@@ -10,6 +10,12 @@
 // Without scores (s = NULL) the call is plain causal GQA attention: the kernel
 // instantiation without the bias step runs (tau = 0 keeps it, with a block of zeros).
 //
+// Two kernels.  When the grid below would hold at most 1.5 CTAs per SM (a short
+// sequence: S = 2560 with 16 heads is 160 CTAs on 148 SMs) the call runs the persistent
+// kernel of attention_persistent.cu instead, one CTA per SM working through single
+// query tiles, which fills the SMs and balances the causal triangle; longer sequences
+// run the kernel below, whose CTAs share each K/V tile between two query tiles.
+//
 // B200 design (flash-style, one CTA per pair of 128-row query tiles of one head):
 //   * TMEM (512 columns): S_0, S_1 (128 fp32 columns each, one per query tile),
 //     O_0, O_1 (D columns each).  The bf16 probabilities P_t are written back over
@@ -57,6 +63,7 @@
 #include <algorithm>
 #include <cmath>
 
+#include "internal.h"
 #include "ptx.cuh"
 #include "runtime.h"
 
@@ -580,6 +587,9 @@ template <int D>
 tg_status launch(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s, const float *gain, float tau,
                  const int32_t *cu_seqlens, int32_t B, int64_t total, int64_t max_seqlen, int32_t Hq, int32_t Hkv,
                  tg_bf16 *O, float *lse, float *O32, cudaStream_t stream, uint32_t *err) {
+  if (tg::attention_uses_persistent(max_seqlen, Hq, B))
+    return tg::gated_attention_persistent(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, D, O,
+                                          lse, O32, stream, err);
   // plain causal attention leaves the bias step out; with tau = 0 it is the whole product
   if (s || tau == 0.f)
     return launch_kernel<D, true>(Q, Kc, V, s, gain, tau, cu_seqlens, B, total, max_seqlen, Hq, Hkv, O, lse, O32,
@@ -605,6 +615,15 @@ tg_status validate(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const 
 }
 
 }  // namespace
+
+namespace tg {
+
+bool attention_uses_persistent(int64_t max_seqlen, int32_t Hq, int32_t B) {
+  const int64_t two_tile_ctas = (max_seqlen + 2 * kBM - 1) / (2 * kBM) * Hq * B;
+  return 2 * two_tile_ctas <= 3 * static_cast<int64_t>(sm_count());
+}
+
+}  // namespace tg
 
 extern "C" tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, const float *s,
                                         const float *gain, float tau, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
