@@ -473,59 +473,212 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // every CTA is past its remote reads
 }
 
-// Varlen pre-pass (one CTA): kept count of every request, min(k_b, n_doc_b) + question_b,
-// then their prefix sums into cu_kept[0..B].  Also validates cu_seqlens.
+// Varlen pre-pass (one CTA of 1024 threads): the kept count of every request,
+// min(k_b, n_doc_b) + question_b, and their prefix sums into cu_kept[0..B]; it also
+// validates cu_seqlens.  For a well-formed batch of at most kSegFast requests one pass
+// over the mask suffices: each thread counts the document tokens of a contiguous run of
+// 16-byte words (the mask's address decides where whole words start; the bytes before
+// and after them are counted singly) and records, for every request boundary inside its
+// run, the count up to that boundary; a block scan of the run counts turns those into
+// the number of document tokens before every boundary, and the differences of
+// consecutive boundaries are the requests' document counts.  A malformed or larger batch
+// takes one request at a time.
+constexpr int kSegFast = 4096;
+
+__device__ __forceinline__ uint32_t doc_bytes(uint32_t w) { return __popc(__vcmpne4(w, 0u)) >> 3; }
+__device__ __forceinline__ uint32_t doc_bytes(const uint4 &v) {
+  return doc_bytes(v.x) + doc_bytes(v.y) + doc_bytes(v.z) + doc_bytes(v.w);
+}
+// document bytes among the first n (0..16) bytes of a 16-byte word
+__device__ __forceinline__ uint32_t doc_bytes_prefix(const uint4 &v, int n) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k = n - 4 * q;  // bytes of this 32-bit lane to count
+    const uint32_t keep = k >= 4 ? 0xFFFFFFFFu : (k <= 0 ? 0u : (0xFFFFFFFFu >> (32 - 8 * k)));
+    c += doc_bytes(w[q] & keep);
+  }
+  return c;
+}
+
+// exclusive scan over the 1024 threads of the block (32 warps); *total gets the sum
+__device__ __forceinline__ uint32_t seg_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = wsum[lane];
+    uint32_t wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, wi, off);
+      if (lane >= off) wi += u;
+    }
+    wsum[lane] = wi - w;
+    if (lane == 31) wsum[32] = wi;
+  }
+  __syncthreads();
+  const uint32_t res = wsum[warp] + incl - v;
+  *total = wsum[32];
+  __syncthreads();  // wsum may be reused by the next scan
+  return res;
+}
+
 __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__restrict__ mask,
                                                            const int32_t *__restrict__ cu_seqlens, int32_t B,
                                                            int64_t total, const int32_t *__restrict__ k_per_seq,
                                                            int32_t *__restrict__ cu_kept, uint32_t *err) {
-  __shared__ long long red[32];
-  __shared__ long long run;
+  __shared__ int32_t s_cu[kSegFast + 1];
+  __shared__ uint32_t s_pre[kSegFast + 1];  // document tokens before each boundary
+  __shared__ uint32_t wsum[33];
+  __shared__ uint32_t s_head;
   tg::pdl_wait();
   tg::pdl_trigger();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    run = 0;
-    cu_kept[0] = 0;
+  const int t = static_cast<int>(threadIdx.x);
+  const int nt = static_cast<int>(blockDim.x);
+  const int lane = t & 31, warp = t >> 5;
+
+  bool bad = false;
+  for (int b = t; b < B; b += nt) {
+    const int64_t s = cu_seqlens[b], e = cu_seqlens[b + 1];
+    bad = bad || s < 0 || e < s || e > total || (b == 0 && s != 0);
+  }
+  if (bad) tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
+  if (t == 0) cu_kept[0] = 0;
+  if (B == 0) return;  // uniform over the block
+  if (__syncthreads_or(bad) || B > kSegFast) {
+    // one request at a time (ranges clamped into [0, total])
+    __shared__ long long red[32];
+    __shared__ long long run;
+    if (t == 0) run = 0;
+    __syncthreads();
+    for (int b = 0; b < B; ++b) {
+      int64_t s = cu_seqlens[b], e = cu_seqlens[b + 1];
+      s = s < 0 ? 0 : (s > total ? total : s);
+      e = e < s ? s : (e > total ? total : e);
+      // whole 16-byte words where the mask's address is aligned, single bytes around them
+      const int64_t a0 = s + static_cast<int64_t>((16u - (reinterpret_cast<uintptr_t>(mask + s) & 15u)) & 15u);
+      long long cnt = 0;
+      if (a0 + 16 <= e) {
+        const int64_t nw = (e - a0) >> 4, a1 = a0 + 16 * nw;
+        const uint4 *w = reinterpret_cast<const uint4 *>(mask + a0);
+        for (int64_t q = t; q < nw; q += nt) cnt += doc_bytes(__ldg(w + q));
+        for (int64_t i = s + t; i < a0; i += nt) cnt += mask[i] != 0;
+        for (int64_t i = a1 + t; i < e; i += nt) cnt += mask[i] != 0;
+      } else {
+        for (int64_t i = s + t; i < e; i += nt) cnt += mask[i] != 0;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) cnt += __shfl_down_sync(0xFFFFFFFFu, cnt, off);
+      if (lane == 0) red[warp] = cnt;
+      __syncthreads();
+      if (t == 0) {
+        long long n_doc = 0;
+        for (int w = 0; w < nt / 32; ++w) n_doc += red[w];
+        long long k = k_per_seq[b];
+        if (k < 0) k = 0;
+        run += (k < n_doc ? k : n_doc) + ((e - s) - n_doc);
+        cu_kept[b + 1] = static_cast<int32_t>(run);
+      }
+      __syncthreads();
+    }
+    return;
+  }
+
+  // ---- one pass: requests cover [0, E), well formed
+  for (int b = t; b <= B; b += nt) s_cu[b] = cu_seqlens[b];
+  __syncthreads();
+  const int64_t E = s_cu[B];
+  const int64_t a_mis = static_cast<int64_t>((16u - (reinterpret_cast<uintptr_t>(mask) & 15u)) & 15u);
+  const int64_t A0 = a_mis < E ? a_mis : E;  // whole words start where the mask's address is aligned
+  const int64_t nw = (E - A0) >> 4, A1 = A0 + 16 * nw;
+  if (warp == 0) {
+    const bool d = lane < A0 && mask[lane] != 0;
+    const uint32_t h = __popc(__ballot_sync(0xFFFFFFFFu, d));
+    if (lane == 0) s_head = h;
+  }
+  // this thread's run of words and the boundaries inside it
+  const int64_t per = (nw + nt - 1) / nt;
+  const int64_t w0 = static_cast<int64_t>(t) * per < nw ? static_cast<int64_t>(t) * per : nw;
+  const int64_t w1 = w0 + per < nw ? w0 + per : nw;
+  int b_first = B + 1;
+  {
+    int lo = 0, hi = B + 1;  // first boundary >= the run's first position
+    const int64_t p0 = A0 + 16 * w0;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (s_cu[mid] < p0) lo = mid + 1;
+      else hi = mid;
+    }
+    b_first = lo;
+  }
+  int b_end = b_first;
+  uint32_t local = 0;
+  const uint4 *mw = reinterpret_cast<const uint4 *>(mask + A0);
+  // eight loads in flight at a time (the run's words are independent)
+  for (int64_t wb = w0; wb < w1; wb += 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = wb + i < w1 ? __ldg(mw + wb + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (wb + i >= w1) break;
+      const int64_t ws = A0 + 16 * (wb + i);
+      while (b_end <= B && s_cu[b_end] < ws + 16) {
+        s_pre[b_end] = local + doc_bytes_prefix(v[i], static_cast<int>(s_cu[b_end] - ws));
+        ++b_end;
+      }
+      local += doc_bytes(v[i]);
+    }
+  }
+  uint32_t words_total;
+  const uint32_t before = seg_excl_scan(local, wsum, &words_total);
+  const uint32_t head = s_head;
+  for (int b = b_first; b < b_end; ++b) s_pre[b] += head + before;
+  // boundaries before the first whole word or at / after the end of the last one
+  for (int b = t; b <= B; b += nt) {
+    const int64_t x = s_cu[b];
+    if (x < A0 || x >= A1) {
+      uint32_t c = 0;
+      if (x < A0) {
+        for (int64_t i = 0; i < x; ++i) c += mask[i] != 0;
+      } else {
+        c = head + words_total;
+        for (int64_t i = A1; i < x; ++i) c += mask[i] != 0;
+      }
+      s_pre[b] = c;
+    }
   }
   __syncthreads();
-  for (int b = 0; b < B; ++b) {
-    int64_t s = cu_seqlens[b], e = cu_seqlens[b + 1];
-    if (threadIdx.x == 0 && (s < 0 || e < s || e > total || (b == 0 && s != 0)))
-      tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
-    s = s < 0 ? 0 : (s > total ? total : s);
-    e = e < s ? s : (e > total ? total : e);
-    // document tokens of the request: 16-byte words over its aligned body (nonzero bytes
-    // counted four at a time), single bytes over the unaligned head and tail
-    long long cnt = 0;
-    const int64_t a0 = (s + 15) & ~int64_t(15), a1 = e & ~int64_t(15);
-    if (a0 < a1) {
-      const uint4 *w = reinterpret_cast<const uint4 *>(mask + a0);
-      const int64_t nw = (a1 - a0) >> 4;
-      for (int64_t q = threadIdx.x; q < nw; q += blockDim.x) {
-        const uint4 v = __ldg(w + q);
-        cnt += (__popc(__vcmpne4(v.x, 0u)) + __popc(__vcmpne4(v.y, 0u)) + __popc(__vcmpne4(v.z, 0u)) +
-                __popc(__vcmpne4(v.w, 0u))) >> 3;
-      }
-      for (int64_t i = s + threadIdx.x; i < a0; i += blockDim.x) cnt += mask[i] != 0;
-      for (int64_t i = a1 + threadIdx.x; i < e; i += blockDim.x) cnt += mask[i] != 0;
-    } else {
-      for (int64_t i = s + threadIdx.x; i < e; i += blockDim.x) cnt += mask[i] != 0;
-    }
+  // kept counts of four consecutive requests per thread, then their prefix sums
+  uint32_t kept[4], sum = 0;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_down_sync(0xFFFFFFFFu, cnt, off);
-    if (lane == 0) red[warp] = cnt;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      long long n_doc = 0;
-      for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) n_doc += red[w];
-      long long k = k_per_seq[b];
-      if (k < 0) k = 0;
-      const long long kept = (k < n_doc ? k : n_doc) + ((e - s) - n_doc);
-      run += kept;
-      cu_kept[b + 1] = static_cast<int32_t>(run);
+  for (int q = 0; q < 4; ++q) {
+    const int b = 4 * t + q;
+    kept[q] = 0;
+    if (b < B) {
+      const uint32_t n_doc = s_pre[b + 1] - s_pre[b];
+      const uint32_t len = static_cast<uint32_t>(s_cu[b + 1] - s_cu[b]);
+      const int32_t kb = k_per_seq[b];
+      const uint32_t k = kb < 0 ? 0u : static_cast<uint32_t>(kb);
+      kept[q] = (k < n_doc ? k : n_doc) + (len - n_doc);
     }
-    __syncthreads();
+    sum += kept[q];
+  }
+  uint32_t all;
+  uint32_t run = seg_excl_scan(sum, wsum, &all);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int b = 4 * t + q;
+    run += kept[q];
+    if (b < B) cu_kept[b + 1] = static_cast<int32_t>(run);
   }
 }
 

@@ -230,6 +230,53 @@ def test_topk_varlen_bit_exact(lens):
     assert bits & ~tg.TG_DEVERR_K_GT_NDOC == 0
 
 
+@pytest.mark.parametrize("offset", [1, 7])
+def test_topk_varlen_unaligned_mask_and_scores(offset):
+    """doc_mask and scores carry no alignment requirement: views that start ``offset``
+    elements into their buffers (the pre-pass then counts the mask's leading bytes singly
+    and takes whole 16-byte words from the first aligned address on)."""
+    lens = [300, 5000, 17, 2048, 0, 999]
+    rng = np.random.default_rng(offset)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    s = W.mixture_scores(total, 9).numpy()
+    mask = (rng.random(total) < 0.9).astype(np.uint8)
+    ks = [int(rng.integers(0, L + 2)) for L in lens]
+    ref, ref_cu = oracle.select_topk_varlen(s, mask, cu, ks)
+    s_buf = torch.zeros(total + offset, dtype=torch.float32, device=DEV)
+    m_buf = torch.zeros(total + offset, dtype=torch.uint8, device=DEV)
+    s_buf[offset:] = torch.as_tensor(s).to(DEV)
+    m_buf[offset:] = torch.as_tensor(mask).to(DEV)
+    kept, cu_kept = tg.tg_select_topk_varlen(s_buf[offset:], m_buf[offset:], torch.as_tensor(cu).to(DEV),
+                                             torch.tensor(ks, dtype=torch.int32).to(DEV), max(lens))
+    cu_kept = cu_kept.cpu().numpy()
+    assert np.array_equal(cu_kept, ref_cu)
+    assert np.array_equal(kept[:cu_kept[-1]].cpu().numpy(), ref)
+    assert _devbits() & ~tg.TG_DEVERR_K_GT_NDOC == 0
+
+
+@pytest.mark.parametrize("B", [3000, 5000])
+def test_topk_varlen_many_short_requests(B):
+    """Thousands of requests of 0-40 tokens: the one-pass pre-pass (up to 4096 requests,
+    many boundaries inside one thread's run of mask words) and the request-at-a-time one
+    above it give the oracle's offsets."""
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 41, size=B)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    s = W.mixture_scores(total, 3).numpy()
+    mask = (rng.random(total) < 0.7).astype(np.uint8)
+    ks = rng.integers(-1, 30, size=B).astype(np.int32)
+    ref, ref_cu = oracle.select_topk_varlen(s, mask, cu, [int(k) for k in ks])
+    kept, cu_kept = tg.tg_select_topk_varlen(torch.as_tensor(s).to(DEV), torch.as_tensor(mask).to(DEV),
+                                             torch.as_tensor(cu).to(DEV), torch.as_tensor(ks).to(DEV),
+                                             int(lens.max()))
+    cu_kept = cu_kept.cpu().numpy()
+    assert np.array_equal(cu_kept, ref_cu)
+    assert np.array_equal(kept[:cu_kept[-1]].cpu().numpy(), ref)
+    assert _devbits() & ~tg.TG_DEVERR_K_GT_NDOC == 0
+
+
 @pytest.mark.parametrize("n", [1, 100, 4097, 131072, 200003])
 def test_random_k_bit_exact(n):
     rng = np.random.default_rng(n + 7)
