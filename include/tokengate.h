@@ -72,7 +72,8 @@ enum {
     TG_DEVERR_INDEX_OOB = 2u,  /* tg_gather met an index outside [0, n); that row was skipped */
     TG_DEVERR_K_GT_NDOC = 4u,  /* budget above the document length; clamped to keep every document token */
     TG_DEVERR_CAPACITY = 8u,   /* kept tokens exceed the output capacity; writes past it were dropped */
-    TG_DEVERR_BAD_SEQLENS = 16u /* cu_seqlens not non-decreasing within [0, total] */
+    TG_DEVERR_BAD_SEQLENS = 16u /* cu_seqlens not non-decreasing within [0, total], or a
+                                   request longer than max_seqlen */
 };
 
 /* ABI version of the loaded library (TG_ABI_VERSION it was built with). */
@@ -265,7 +266,10 @@ tg_status tg_gated_attention_train(const tg_bf16 *Q, const tg_bf16 *Kc, const tg
  * Q, Kc, V, s and O (cu_seqlens: device int32 [B+1], e.g. cu_kept from
  * tg_select_topk_varlen) and attends causally within itself only.  total is
  * the packed row count and max_seqlen a host upper bound on any request's
- * length (it sizes the grid). */
+ * length (it sizes the grid).  A range outside [0, total], a decreasing one or a
+ * request with rows beyond those max_seqlen covers (rounded up to whole tiles) sets
+ * TG_DEVERR_BAD_SEQLENS (that request's output is then incomplete; the ranges are
+ * clamped into [0, total]). */
 tg_status tg_gated_attention_varlen(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
                                     const float *s, const float *gain, float tau,
                                     const int32_t *cu_seqlens, int32_t B, int64_t total,

@@ -142,6 +142,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t seg_start = 0, len = S_single;
   if (cu_seqlens) {
     int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
+    // one CTA per request reports a malformed range or a request past the grid's rows
+    // (longer than max_seqlen), whose remaining rows no CTA computes
+    if (threadIdx.x == 0 && h == 0 && mb == n_mblocks - 1 &&
+        (s0 < 0 || s1 < s0 || s1 > total || s1 - s0 > static_cast<int64_t>(n_mblocks) * 2 * kBM))
+      tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
     s0 = s0 < 0 ? 0 : (s0 > total ? total : s0);
     s1 = s1 < s0 ? s0 : (s1 > total ? total : s1);
     seg_start = s0;

@@ -563,6 +563,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const bool leader = (warp == 12 && lane == 0);
+    // CTA 0 reports a malformed request range or a request past the grid's rows (longer
+    // than max_seqlen), whose remaining rows no item covers
+    if (cu_seqlens && blockIdx.x == 0 && warp == 12) {
+      for (int b = lane; b < B; b += 32) {
+        const int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
+        if (s0 < 0 || s1 < s0 || s1 > total || s1 - s0 > static_cast<int64_t>(n_mt) * kBM)
+          tg::set_device_error(err, TG_DEVERR_BAD_SEQLENS);
+      }
+    }
     auto load_q = [&](const Item &qi, int buf) {
       const uint32_t q_taddr = tmem_base + C::kTmemQ + static_cast<uint32_t>(buf * (D / 2)) + lane_off;
       const int64_t row = qi.rt + r;

@@ -152,3 +152,22 @@ def test_training_forward_varlen_on_both_kernels(kernel):
                       torch.as_tensor(cu).to(DEV), max(lens), max_seqlen=max(lens), B=len(lens))
     check_attention(O.float().numpy(), Q, K, V, s, gain, 1.1, cu=cu)
     check_attention(O32.numpy(), Q, K, V, s, gain, 1.1, cu=cu, fp32_out=True)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_varlen_request_past_max_seqlen_sets_the_status_bit(kernel):
+    """A request longer than the rows max_seqlen covers is reported, not silently cut; a
+    well-formed call afterwards is clean."""
+    lens = [300, 1000]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Q, K, V, s, gain = _attn_inputs(int(cu[-1]), 4, 2, 128, 12)
+    r = replication_for(kernel, 100, 4, B=2)  # the kernel the bad call (max_seqlen 100) runs; the good one runs it too
+    Qr, Kr, Vr, gr = tile_heads(r, Q, K, V, gain)
+    d_cu = torch.as_tensor(cu).to(DEV)
+    tg.tg_get_device_error()
+    tg.tg_gated_attention_varlen(Qr.to(DEV), Kr.to(DEV), Vr.to(DEV), s.to(DEV), gr.to(DEV), 1.1, d_cu, 100)
+    torch.cuda.synchronize()
+    assert tg.tg_get_device_error() & tg.TG_DEVERR_BAD_SEQLENS
+    tg.tg_gated_attention_varlen(Qr.to(DEV), Kr.to(DEV), Vr.to(DEV), s.to(DEV), gr.to(DEV), 1.1, d_cu, 1000)
+    torch.cuda.synchronize()
+    assert tg.tg_get_device_error() == 0
