@@ -9,7 +9,8 @@
 // (cp.async.bulk global->shared with mbarrier completion, then
 // cp.async.bulk shared->global), so no thread touches the payload.  Each warp
 // runs its own pipeline of ``stages`` row buffers; one lane issues the copies.
-// The grid is sized to two CTAs per SM, keeping several MB of copies in flight.
+// The grid is sized to two CTAs per SM (fewer only when there are fewer rows than
+// warps), keeping several MB of copies in flight.
 #include <algorithm>
 
 #include "ptx.cuh"
@@ -125,8 +126,9 @@ extern "C" tg_status tg_gather(const tg_bf16 *hidden, int64_t n, int32_t d, cons
         cudaFuncSetAttribute(gather_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   }
-  const int64_t warps_needed = (n_rows + stages - 1) / stages;
-  int64_t grid = (warps_needed + kWarps - 1) / kWarps;
+  // one row per warp before any warp takes a second, so that a short gather still spreads
+  // over every SM (up to two CTAs per SM)
+  int64_t grid = (n_rows + kWarps - 1) / kWarps;
   grid = std::max<int64_t>(1, std::min<int64_t>(grid, 2LL * tg::sm_count()));
   const cudaError_t e = tg::launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
                                       static_cast<cudaStream_t>(stream), reinterpret_cast<const uint8_t *>(hidden), n,

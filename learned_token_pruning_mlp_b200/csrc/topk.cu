@@ -8,7 +8,8 @@
 //
 // B200 design: the work is memory-trivial (5 bytes a token), so the cost is
 // latency.  One request is handled by one 8-CTA thread-block cluster of 1024
-// threads each; every thread owns 16 consecutive positions (loaded with 16-byte
+// threads each (a request of at most 8192 positions by one CTA alone, the same code
+// with a cluster of one); every thread owns 16 consecutive positions (loaded with 16-byte
 // vector loads) and keeps their 32-bit order keys in registers (131072 positions per
 // cluster; longer requests re-derive the keys from the scores on every pass).  Up to
 // three radix passes over 11-, 11- and 10-bit digits find the K-th largest key (each
@@ -20,9 +21,9 @@
 // whose chosen bin holds exactly the keys still needed ends the search early.
 // Histograms alternate between two buffers, so one barrier per pass suffices.  When
 // the first digit's histogram comes precomputed (tg_select_fused: the gate's epilogue
-// counts the top 8 bits), the passes use four 8-bit digits instead.  The ordered compaction needs one scan of packed (tie, keep) counts
-// per CTA and one exchange of the per-CTA totals.  No workspace, no global atomics,
-// one launch for a single request.
+// counts the top 8 bits), the passes use four 8-bit digits instead.  The ordered
+// compaction needs one scan of packed (tie, keep) counts per CTA and one exchange of the
+// per-CTA totals.  No workspace, no global atomics, one launch for a single request.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -36,7 +37,7 @@ namespace cg = cooperative_groups;
 
 namespace {
 
-constexpr int kCluster = 8;
+constexpr int kCluster = 8;                       // CTAs per request above kRound positions
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kItems = 16;                        // consecutive positions per thread
@@ -103,6 +104,7 @@ __device__ __forceinline__ void fold_coarse(TopkShared &sh, int buf, int nbins) 
 // of that coarse bin are summed over the eight CTAs.  Publishes sel_digit, sel_above
 // (candidates in higher bins) and sel_count (candidates in the chosen bin);
 // sel_digit = nbins if none qualifies.  The total lands in wsum[kWarps].
+template <int kC>
 __device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster, TopkShared &sh, int buf,
                                                      int nbins, uint32_t remaining) {
   const int g = nbins / kCoarse;
@@ -111,7 +113,7 @@ __device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster,
   uint32_t cnt = 0;
   if (t < kCoarse) {
 #pragma unroll
-    for (int r = 0; r < kCluster; ++r) cnt += cluster.map_shared_rank(&sh.coarse[buf][0], r)[cb];
+    for (int r = 0; r < kC; ++r) cnt += cluster.map_shared_rank(&sh.coarse[buf][0], r)[cb];
   }
   if (t == 0) sh.sel_digit = nbins;  // ordered before the writes below by the scan's barriers
   uint32_t total;
@@ -124,14 +126,14 @@ __device__ __forceinline__ void cluster_select_digit(cg::cluster_group &cluster,
   }
   __syncthreads();
   if (g == 1 || sh.sel_digit != static_cast<uint32_t>(nbins) || remaining == 0 || remaining > total) return;
-  // the fine bins of the chosen coarse bin: lane group j (8 lanes, one per CTA) sums fine
-  // bin cbin * g + g - 1 - j
+  // the fine bins of the chosen coarse bin: lane group j (kC lanes, one per CTA) sums
+  // fine bin cbin * g + g - 1 - j
   const uint32_t cbin = sh.sel_cbin;
-  if (t < 8 * g) {
-    const int j = t >> 3, r = t & 7;
+  if (t < kC * g) {
+    const int j = t / kC, r = t % kC;
     uint32_t c = cluster.map_shared_rank(&sh.hist[buf][0], r)[cbin * g + g - 1 - j];
 #pragma unroll
-    for (int off = 4; off > 0; off >>= 1) c += __shfl_down_sync(0xFFFFFFFFu, c, off, 8);
+    for (int off = kC / 2; off > 0; off >>= 1) c += __shfl_down_sync(0xFFFFFFFFu, c, off, kC);
     if (r == 0) sh.fine[j] = c;
   }
   __syncthreads();
@@ -197,15 +199,17 @@ __device__ __forceinline__ uint32_t random_key(uint64_t seed, int64_t pos, bool 
 // selects from [0, n_single) with its own budget k_sweep[b] into its own output block.
 // kResident: every CTA's chunk fits one round (<= 16384 positions), keys stay in
 // registers; otherwise the keys are re-derived from the scores on every pass.
-template <bool kResident>
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+// kC: CTAs per cluster, 8, or 1 when a request fits one CTA's registers (no cluster
+// barrier or distributed-shared-memory read is then paid).
+template <bool kResident, int kC>
+__global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 1)
     topk_cluster_kernel(const TopkArgs args) {
   __shared__ TopkShared sh;
   tg::pdl_wait();
   tg::pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int seg = static_cast<int>(blockIdx.x) / kCluster;
+  const int seg = static_cast<int>(blockIdx.x) / kC;
   const float *__restrict__ scores = args.scores;
   const uint8_t *__restrict__ mask = args.mask;
   const int32_t *__restrict__ cu_seqlens = args.cu_seqlens;
@@ -231,7 +235,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   if (k < 0) k = 0;
   const int64_t len = end - start;
   // chunk: a multiple of kItems so that a thread's positions never straddle two CTAs
-  const int64_t chunk = ((len + kCluster - 1) / kCluster + kItems - 1) / kItems * kItems;
+  const int64_t chunk = ((len + kC - 1) / kC + kItems - 1) / kItems * kItems;
   const int64_t lo = start + chunk * rank;
   const int64_t hi = lo + chunk < end ? lo + chunk : end;
   const int m = lo < hi ? static_cast<int>(hi - lo) : 0;
@@ -310,7 +314,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       // CTA's share of its partial histograms (the cluster reduction adds the shares)
       if (threadIdx.x < kPassBins8) {
         uint32_t c = 0;
-        for (int p = rank; p < args.n_parts; p += kCluster)
+        for (int p = rank; p < args.n_parts; p += kC)
           c += __ldg(args.hist_parts + p * kPassBins8 + threadIdx.x);
         sh.hist[0][threadIdx.x] = c;
       }
@@ -326,7 +330,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     fold_coarse(sh, buf, nbins);
     __syncthreads();
     cluster.sync();
-    cluster_select_digit(cluster, sh, buf, nbins, remaining);
+    cluster_select_digit<kC>(cluster, sh, buf, nbins, remaining);
     if (pass == 0) {
       n_doc = sh.wsum[kWarps];
       if (k > n_doc && rank == 0 && threadIdx.x == 0) tg::set_device_error(err, TG_DEVERR_K_GT_NDOC);
@@ -392,28 +396,28 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     // lane r < 8 reads CTA r's counts; the prefixes over CTAs come from warp shuffles
     const int lane = threadIdx.x;
     long long eq = 0, gtq = 0;
-    if (lane < kCluster) {
+    if (lane < kC) {
       const long long *x = cluster.map_shared_rank(&sh.exch[0], lane);
       eq = x[0];
       gtq = x[1];
     }
     long long eq_incl = eq;
 #pragma unroll
-    for (int off = 1; off < kCluster; off <<= 1) {
+    for (int off = 1; off < kC; off <<= 1) {
       const long long t = __shfl_up_sync(0xFFFFFFFFu, eq_incl, off);
       if (lane >= off) eq_incl += t;
     }
     const long long tb = eq_incl - eq;  // ties in CTAs before this lane's CTA
     long long th = need_eq - tb;
     th = th < 0 ? 0 : (th > eq ? eq : th);
-    const long long keep = lane < kCluster ? gtq + th : 0;
+    const long long keep = lane < kC ? gtq + th : 0;
     long long keep_incl = keep;
 #pragma unroll
-    for (int off = 1; off < kCluster; off <<= 1) {
+    for (int off = 1; off < kC; off <<= 1) {
       const long long t = __shfl_up_sync(0xFFFFFFFFu, keep_incl, off);
       if (lane >= off) keep_incl += t;
     }
-    const long long nt = __shfl_sync(0xFFFFFFFFu, keep_incl, kCluster - 1);
+    const long long nt = __shfl_sync(0xFFFFFFFFu, keep_incl, kC - 1);
     if (lane == rank) {
       sh.bcast[0] = tb;
       sh.bcast[1] = base + keep_incl - keep;
@@ -682,13 +686,26 @@ __global__ void __launch_bounds__(1024) seg_offsets_kernel(const uint8_t *__rest
   }
 }
 
-cudaError_t launch_cluster(bool resident, unsigned grid, cudaStream_t s, const TopkArgs &a) {
-  if (resident) return tg::launch_pdl(topk_cluster_kernel<true>, dim3(grid), dim3(kThreads), 0, s, a);
-  return tg::launch_pdl(topk_cluster_kernel<false>, dim3(grid), dim3(kThreads), 0, s, a);
-}
+// CTAs per request for requests of at most ``len`` positions: one for up to half a
+// CTA's register tile (measured: 4096 positions 11.5 us against 12.5 us in a cluster,
+// 16384 positions 13.1 us against 12.6 us), else a cluster of kCluster
+constexpr int64_t kLoneCta = kRound / 2;
+int cluster_for(int64_t len) { return len <= kLoneCta ? 1 : kCluster; }
 
-// chunk per CTA for a request of ``len`` positions (as the kernel computes it)
-int64_t chunk_of(int64_t len) { return ((len + kCluster - 1) / kCluster + kItems - 1) / kItems * kItems; }
+// chunk per CTA for a request of ``len`` positions in clusters of kc CTAs (as the kernel
+// computes it)
+int64_t chunk_of(int64_t len, int kc) { return ((len + kc - 1) / kc + kItems - 1) / kItems * kItems; }
+
+// ``n_seg`` clusters (requests, or budgets in sweep mode) of cluster_for(len_bound) CTAs
+cudaError_t launch_cluster(int64_t len_bound, unsigned n_seg, cudaStream_t s, const TopkArgs &a) {
+  const int kc = cluster_for(len_bound);
+  const bool resident = chunk_of(len_bound, kc) <= kRound;
+  const dim3 grid(n_seg * static_cast<unsigned>(kc));
+  // a lone CTA always holds its request in registers (len_bound <= kLoneCta < kRound)
+  if (kc == 1) return tg::launch_pdl(topk_cluster_kernel<true, 1>, grid, dim3(kThreads), 0, s, a);
+  if (resident) return tg::launch_pdl(topk_cluster_kernel<true, kCluster>, grid, dim3(kThreads), 0, s, a);
+  return tg::launch_pdl(topk_cluster_kernel<false, kCluster>, grid, dim3(kThreads), 0, s, a);
+}
 
 }  // namespace
 
@@ -713,7 +730,7 @@ extern "C" tg_status tg_select_topk(const float *scores, const uint8_t *doc_mask
   a.cap = cap;
   a.n_kept = n_kept;
   a.err = err;
-  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
+  const cudaError_t e = launch_cluster(n, 1, static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
@@ -742,7 +759,7 @@ tg_status tg::select_topk_hist(const float *scores, const uint8_t *doc_mask, int
   a.hist_parts = hist_parts;
   a.n_parts = n_parts;
   a.err = err;
-  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
+  const cudaError_t e = launch_cluster(n, 1, static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
@@ -769,7 +786,7 @@ extern "C" tg_status tg_select_random_k(const uint8_t *doc_mask, int64_t n, int6
   a.seed = seed;
   a.random = 1;
   a.err = err;
-  const cudaError_t e = launch_cluster(chunk_of(n) <= kRound, kCluster, static_cast<cudaStream_t>(stream), a);
+  const cudaError_t e = launch_cluster(n, 1, static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
@@ -800,7 +817,7 @@ extern "C" tg_status tg_select_topk_sweep(const float *scores, const uint8_t *do
   a.n_kept = n_kept;
   a.err = err;
   const cudaError_t e =
-      launch_cluster(chunk_of(n) <= kRound, static_cast<unsigned>(m) * kCluster, static_cast<cudaStream_t>(stream), a);
+      launch_cluster(n, static_cast<unsigned>(m), static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
@@ -837,7 +854,7 @@ extern "C" tg_status tg_select_topk_varlen(const float *scores, const uint8_t *d
   a.err = err;
   // the register-resident variant is chosen when max_seqlen fits it; a request longer
   // than max_seqlen then sets TG_DEVERR_BAD_SEQLENS
-  e = launch_cluster(chunk_of(max_seqlen) <= kRound, static_cast<unsigned>(B) * kCluster, s, a);
+  e = launch_cluster(max_seqlen, static_cast<unsigned>(B), s, a);
   if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "topk_cluster_kernel launch: %s", cudaGetErrorString(e));
   return tg::check_launch("topk_cluster_kernel");
 }
