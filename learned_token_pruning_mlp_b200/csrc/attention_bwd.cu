@@ -22,7 +22,7 @@
 //      queries is a register sum.  Per 128-query block, from the diagonal on:
 //          S^T  = K Q^T    and    dP^T = V dO^T
 //      (tcgen05, M = 128 keys, N = 128 queries, K = D, operands K-major in shared
-//      memory) go to one of two TMEM buffers while two warpgroups (64 query columns
+//      memory) go to one of two TMEM buffers while four warpgroups (32 query columns
 //      each) form p = exp2(S c + b_j - lse2_i) with c = tau log2(e) / sqrt(D) and
 //      b_j = gain_h log2(e) s_j, dl = p (dP - Delta_i), and accumulate sum_i dl and
 //      sum_i dl S with packed f32x2 arithmetic.  Q and dO stream through a TMA
@@ -44,7 +44,7 @@ namespace {
 
 constexpr int kBK = 128;          // keys per CTA (TMEM lanes)
 constexpr int kBQ = 128;          // queries per step (TMEM columns of S^T and dP^T)
-constexpr int kThreads = 384;     // warps 0-3: TMA, MMA, TMEM alloc, idle; 4-11: two warpgroups
+constexpr int kThreads = 640;     // warps 0-3: TMA, MMA, TMEM alloc, idle; 4-19: four warpgroups
 constexpr int kAux = 4;           // stages of the lse / Delta vectors
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;  // 128 rows x 64 bf16 columns, 128-byte swizzle
@@ -55,7 +55,7 @@ struct BwdCfg {
   static constexpr uint32_t kTileBytes = kHalfBytes * kHalves;  // 128 rows x D bf16
   static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr size_t kSmem = 1024 + 2 * static_cast<size_t>(kTileBytes) +
-                                  2 * static_cast<size_t>(kStages) * kTileBytes + kAux * 2 * kBQ * 4 + kBK * 4 + 512;
+                                  2 * static_cast<size_t>(kStages) * kTileBytes + kAux * 2 * kBQ * 4 + 3 * kBK * 4 + 512;
 };
 
 struct BwdCtl {
@@ -69,7 +69,7 @@ struct BwdCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float tau_part[8];
+  float tau_part[16];
 };
 
 // Workspace (fp32), ``stride`` rows per head (a multiple of 128): -lse2 [Hq][stride],
@@ -228,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sdO = sQ + NS * C::kTileBytes;            // [NS][tile]
   float *sL = reinterpret_cast<float *>(sdO + NS * C::kTileBytes);  // [kAux][kBQ]  -lse2
   float *sDl = sL + kAux * kBQ;                                      // [kAux][kBQ]  -Delta
-  float *sCs = sDl + kAux * kBQ;                                     // [kBK] second warpgroup's column sums
-  BwdCtl *ctl = reinterpret_cast<BwdCtl *>(sCs + kBK);
+  float *sCs = sDl + kAux * kBQ;                                     // [3][kBK] warpgroups 1-3's column sums
+  BwdCtl *ctl = reinterpret_cast<BwdCtl *>(sCs + 3 * kBK);
 
   // (key block, request, head); key blocks ascending: the longest ones first
   const int per_kb = sg.B * Hq;
@@ -254,11 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < kAux; ++a) {
       tg::mbar_init(tg::smem_addr(&ctl->aux_full[a]), 1);
-      tg::mbar_init(tg::smem_addr(&ctl->aux_empty[a]), 8);
+      tg::mbar_init(tg::smem_addr(&ctl->aux_empty[a]), 16);
     }
     for (int b = 0; b < 2; ++b) {
       tg::mbar_init(tg::smem_addr(&ctl->s_full[b]), 1);
-      tg::mbar_init(tg::smem_addr(&ctl->tmem_empty[b]), 256);
+      tg::mbar_init(tg::smem_addr(&ctl->tmem_empty[b]), 512);
     }
     tg::mbar_init(tg::smem_addr(&ctl->drain), 1);
     ctl->abort_flag = 0;
@@ -280,11 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int *abort_flag = &ctl->abort_flag;
 
-  // Register split: the launch gives 384 threads x 168 registers; 128 x 80 + 256 x 208 =
-  // 63488 <= 384 x 168, so the increase never waits (the launcher checks the launch
-  // count).  Each warpgroup changes its budget inside its own branch.
+  // 640 threads at 96 registers each: a dl thread holds 32 columns of S^T and of dP^T,
+  // so no warpgroup needs more than the launch gives (four warpgroups per step keep
+  // four dl warps on every SM sub-partition to hide the exponentials' latency).
   if (warp < 4) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA / bulk producer
     const uint32_t kvb = tg::smem_addr(&ctl->kv_full);
@@ -356,9 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
     // ------------------------------------------------------------ dl and its sums
-    const int grp = (warp - 4) >> 2;       // query columns 64*grp .. 64*grp+63
+    const int grp = (warp - 4) >> 2;       // query columns 32*grp .. 32*grp+31
     const int quarter = warp & 3;          // TMEM lane quarter
     const int r = quarter * 32 + lane;     // key within the block
     const int64_t j = static_cast<int64_t>(kb) * kBK + r;  // request-relative key
@@ -373,26 +371,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->s_full[buf]), (n >> 1) & 1, abort_flag)) break;
       if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->aux_full[a]), (n / kAux) & 1, abort_flag)) break;
       tg::tc_fence_after();
-      const uint32_t t_s = tmem_base + static_cast<uint32_t>(buf * 256 + 64 * grp) + lane_off;
-      uint32_t sx[64], dp[64];
-      tg::tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sx[0]));
-      tg::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sx[32]));
-      tg::tmem_ld32(t_s + kBQ, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-      tg::tmem_ld32(t_s + kBQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      const uint32_t t_s = tmem_base + static_cast<uint32_t>(buf * 256 + 32 * grp) + lane_off;
+      uint32_t sx[32], dp[32];
+      tg::tmem_ld32(t_s, sx);
+      tg::tmem_ld32(t_s + kBQ, dp);
       tg::tmem_ld_wait();
       tg::tc_fence_before();
       tg::mbar_arrive(tg::smem_addr(&ctl->tmem_empty[buf]));
-      const uint64_t *nl = reinterpret_cast<const uint64_t *>(sL + a * kBQ + 64 * grp);
-      const uint64_t *nd = reinterpret_cast<const uint64_t *>(sDl + a * kBQ + 64 * grp);
+      const uint64_t *nl = reinterpret_cast<const uint64_t *>(sL + a * kBQ + 32 * grp);
+      const uint64_t *nd = reinterpret_cast<const uint64_t *>(sDl + a * kBQ + 32 * grp);
       const bool diag = n == 0;  // query block == key block: keep query >= key
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < 16; ++c) {
         const uint64_t s2 = tg::f2_pack(__uint_as_float(sx[2 * c]), __uint_as_float(sx[2 * c + 1]));
         const uint64_t x2 = tg::f2_fma(s2, c2, tg::f2_add(bj2, nl[c]));
         float x0, x1;
         tg::f2_unpack(x2, x0, x1);
         if (diag) {
-          const int q0 = 64 * grp + 2 * c;
+          const int q0 = 32 * grp + 2 * c;
           if (q0 < r) x0 = -INFINITY;
           if (q0 + 1 < r) x1 = -INFINITY;
         }
@@ -410,17 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::f2_unpack(ta2, ta0, ta1);
     float colsum = cs0 + cs1;
     float tacc = ta0 + ta1;
-    if (grp == 1) sCs[r] = colsum;
+    if (grp > 0) sCs[(grp - 1) * kBK + r] = colsum;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) tacc += __shfl_xor_sync(0xFFFFFFFFu, tacc, off);
     if (lane == 0) ctl->tau_part[warp - 4] = tacc;
-    asm volatile("bar.sync 1, 256;" ::: "memory");  // the two warpgroups
+    asm volatile("bar.sync 1, 512;" ::: "memory");  // the four warpgroups
     if (grp == 0) {
-      ws.colsum[wrow0 + j] = colsum + sCs[r];
+      ws.colsum[wrow0 + j] = ((colsum + sCs[r]) + sCs[kBK + r]) + sCs[2 * kBK + r];
       if (r == 0) {
         float t = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) t += ctl->tau_part[w];
+        for (int w = 0; w < 16; ++w) t += ctl->tau_part[w];
         ws.taup[h * (ws.stride / kBK) + sgm.p0 / kBK + kb] = t;
       }
     }
@@ -519,13 +515,6 @@ tg_status launch_bwd(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V, cons
     const cudaError_t e =
         cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    // the warpgroup register split in the kernel assumes 168 registers per thread at launch
-    cudaFuncAttributes fa;
-    const cudaError_t ea = cudaFuncGetAttributes(&fa, attn_bwd_kernel<D>);
-    if (ea != cudaSuccess) return tg::fail(TG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(ea));
-    if (fa.numRegs != 168)
-      return tg::fail(TG_ERR_UNSUPPORTED, "attn_bwd_kernel built with %d registers per thread; the register split "
-                      "needs 168", fa.numRegs);
     return TG_OK;
   });
   if (setup != TG_OK) return setup;
