@@ -25,7 +25,9 @@
 //      memory) go to one of two TMEM buffers while four warpgroups (32 query columns
 //      each) form p = exp2(S c + b_j - lse2_i) with c = tau log2(e) / sqrt(D) and
 //      b_j = gain_h log2(e) s_j, dl = p (dP - Delta_i), and accumulate sum_i dl and
-//      sum_i dl S with packed f32x2 arithmetic.  Q and dO stream through a TMA
+//      sum_i dl S with packed f32x2 arithmetic.  dP - Delta_i comes out of the tensor
+//      core: one extra K step multiplies a block of ones on V's side by -Delta_i in three
+//      bf16 parts on dO's side (written per step by warp 3 from the prep's vector).  Q and dO stream through a TMA
 //      pipeline, the lse / Delta vectors through bulk copies.
 //   3. reduce: ds, dgain and dtau from the per-(head, key) column sums and the
 //      per-CTA temperature partials, each summed in a fixed order, so the result is
@@ -44,10 +46,13 @@ namespace {
 
 constexpr int kBK = 128;          // keys per CTA (TMEM lanes)
 constexpr int kBQ = 128;          // queries per step (TMEM columns of S^T and dP^T)
-constexpr int kThreads = 640;     // warps 0-3: TMA, MMA, TMEM alloc, idle; 4-19: four warpgroups
+constexpr int kThreads = 640;     // warps 0-3: TMA, MMA, TMEM alloc, -Delta blocks; 4-19: four warpgroups
 constexpr int kAux = 4;           // stages of the lse / Delta vectors
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;  // 128 rows x 64 bf16 columns, 128-byte swizzle
+constexpr uint32_t kExtBytes = 128 * 16 * 2;   // one 128-row x 16-column unswizzled block (4 KB)
+constexpr uint32_t kExtLBO = kExtBytes / 2;    // columns 8..15 follow columns 0..7
+constexpr uint32_t kExtSBO = 128;              // 8 rows x 16 bytes per core matrix
 
 template <int D>
 struct BwdCfg {
@@ -55,13 +60,15 @@ struct BwdCfg {
   static constexpr uint32_t kTileBytes = kHalfBytes * kHalves;  // 128 rows x D bf16
   static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr size_t kSmem = 1024 + 2 * static_cast<size_t>(kTileBytes) +
-                                  2 * static_cast<size_t>(kStages) * kTileBytes + kAux * 2 * kBQ * 4 + 3 * kBK * 4 + 512;
+                                  2 * static_cast<size_t>(kStages) * kTileBytes + (1 + kStages) * static_cast<size_t>(kExtBytes) +
+                                  kAux * 2 * kBQ * 4 + 3 * kBK * 4 + 512;
 };
 
 struct BwdCtl {
   uint64_t kv_full;
   uint64_t q_full[4];
   uint64_t q_empty[4];
+  uint64_t ext_full[4];   // the -Delta block of Q / dO stage s is written
   uint64_t aux_full[kAux];
   uint64_t aux_empty[kAux];
   uint64_t s_full[2];
@@ -226,7 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sV = sK + C::kTileBytes;
   uint8_t *sQ = sV + C::kTileBytes;                  // [NS][tile]
   uint8_t *sdO = sQ + NS * C::kTileBytes;            // [NS][tile]
-  float *sL = reinterpret_cast<float *>(sdO + NS * C::kTileBytes);  // [kAux][kBQ]  -lse2
+  uint8_t *sVx = sdO + NS * C::kTileBytes;          // [128 x 16]: ones in columns 0..2 (V's extra K step)
+  uint8_t *sDx = sVx + kExtBytes;                    // [NS][128 x 16]: -Delta in three bf16 parts (dO's)
+  float *sL = reinterpret_cast<float *>(sDx + NS * kExtBytes);      // [kAux][kBQ]  -lse2
   float *sDl = sL + kAux * kBQ;                                      // [kAux][kBQ]  -Delta
   float *sCs = sDl + kAux * kBQ;                                     // [3][kBK] warpgroups 1-3's column sums
   BwdCtl *ctl = reinterpret_cast<BwdCtl *>(sCs + 3 * kBK);
@@ -246,15 +255,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tg::warp_id();
   const int lane = threadIdx.x & 31;
 
+  // V's extra K step: ones in columns 0..2 of every row (bf16 1.0 = 0x3F80), zeros
+  // elsewhere, also in dO's blocks (their columns 0..2 are written per step)
+  for (uint32_t w = threadIdx.x; w < (1 + NS) * kExtBytes / 4; w += kThreads) {
+    uint32_t v = 0;
+    if (w < kExtLBO / 4 && (w & 3u) == 0) v = 0x3F803F80u;
+    if (w < kExtLBO / 4 && (w & 3u) == 1) v = 0x00003F80u;
+    reinterpret_cast<uint32_t *>(sVx)[w] = v;
+  }
+  tg::fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     tg::mbar_init(tg::smem_addr(&ctl->kv_full), 1);
     for (int s = 0; s < NS; ++s) {
       tg::mbar_init(tg::smem_addr(&ctl->q_full[s]), 1);
       tg::mbar_init(tg::smem_addr(&ctl->q_empty[s]), 1);
+      tg::mbar_init(tg::smem_addr(&ctl->ext_full[s]), 1);
     }
     for (int a = 0; a < kAux; ++a) {
       tg::mbar_init(tg::smem_addr(&ctl->aux_full[a]), 1);
-      tg::mbar_init(tg::smem_addr(&ctl->aux_empty[a]), 16);
+      tg::mbar_init(tg::smem_addr(&ctl->aux_empty[a]), 17);  // 16 dl warps and the -Delta block writer
     }
     for (int b = 0; b < 2; ++b) {
       tg::mbar_init(tg::smem_addr(&ctl->s_full[b]), 1);
@@ -312,6 +331,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::bulk_load(tg::smem_addr(sL + a * kBQ), ws.nlse2 + wrow0 + qblk, kBQ * 4, af);
       tg::bulk_load(tg::smem_addr(sDl + a * kBQ), ws.ndelta + wrow0 + qblk, kBQ * 4, af);
     }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ -Delta blocks
+    // dP^T - Delta comes out of the tensor core: one extra K step multiplies V's block of
+    // ones by dO's block holding each query's -Delta split into three bf16 parts (their
+    // sum is -Delta to 2^-24), so the dl loop reads dP - Delta directly.
+    for (int n = 0; n < n_steps; ++n) {
+      const int s = n % NS, a = n % kAux;
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->q_empty[s]), ((n / NS) & 1) ^ 1, abort_flag)) break;
+      if (!tg::mbar_wait_warp(tg::smem_addr(&ctl->aux_full[a]), (n / kAux) & 1, abort_flag)) break;
+#pragma unroll
+      for (int e = 0; e < kBQ / 32; ++e) {
+        const int q = e * 32 + lane;
+        const float v = sDl[a * kBQ + q];
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+        uint8_t *row = sDx + s * kExtBytes + q * 16;  // row q, columns 0..2
+        *reinterpret_cast<__nv_bfloat162 *>(row) = __halves2bfloat162(p0, p1);
+        *reinterpret_cast<__nv_bfloat16 *>(row + 4) = p2;
+      }
+      tg::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tg::mbar_arrive(tg::smem_addr(&ctl->ext_full[s]));
+        tg::mbar_arrive(tg::smem_addr(&ctl->aux_empty[a]));
+      }
+    }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = tg::idesc_bf16_f32(kBK, kBQ, false, false);
@@ -323,6 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t v_lo = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sV), 16, 1024));
     const uint32_t q_lo0 = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sQ), 16, 1024));
     const uint32_t do_lo0 = static_cast<uint32_t>(tg::smem_desc_sw128(tg::smem_addr(sdO), 16, 1024));
+    const uint64_t dvx = tg::smem_desc_noswz(tg::smem_addr(sVx), kExtLBO, kExtSBO);
+    const uint64_t ddx = tg::smem_desc_noswz(tg::smem_addr(sDx), kExtLBO, kExtSBO);
+    const uint32_t dx_lo0 = static_cast<uint32_t>(ddx), hi_x = static_cast<uint32_t>(ddx >> 32);
     constexpr uint32_t kTileUnits = C::kTileBytes >> 4;
     bool ok = tg::mbar_wait(tg::smem_addr(&ctl->kv_full), 0, abort_flag);
     for (int n = 0; n < n_steps && ok; ++n) {
@@ -330,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = n & 1;
       if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->q_full[s]), (n / NS) & 1, abort_flag))) break;
       if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->tmem_empty[buf]), ((n >> 1) & 1) ^ 1, abort_flag))) break;
+      if (!(ok = tg::mbar_wait(tg::smem_addr(&ctl->ext_full[s]), (n / NS) & 1, abort_flag))) break;
       tg::tc_fence_after();
       const uint32_t d_s = tmem_base + static_cast<uint32_t>(buf * 256);
       const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(s) * kTileUnits;
@@ -345,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tg::mma_bf16_ss(d_s + kBQ, tg::desc_words(v_lo + off, hi), tg::desc_words(do_lo + off, hi), idesc,
                         kk > 0 ? 1u : 0u);
       }
+      tg::mma_bf16_ss(d_s + kBQ, dvx, tg::desc_words(dx_lo0 + static_cast<uint32_t>(s) * (kExtBytes >> 4), hi_x), idesc, 1u);
       tg::mma_commit(tg::smem_addr(&ctl->s_full[buf]));
       tg::mma_commit(tg::smem_addr(&ctl->q_empty[s]));
     }
@@ -379,7 +431,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::tc_fence_before();
       tg::mbar_arrive(tg::smem_addr(&ctl->tmem_empty[buf]));
       const uint64_t *nl = reinterpret_cast<const uint64_t *>(sL + a * kBQ + 32 * grp);
-      const uint64_t *nd = reinterpret_cast<const uint64_t *>(sDl + a * kBQ + 32 * grp);
       const bool diag = n == 0;  // query block == key block: keep query >= key
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
@@ -393,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q0 + 1 < r) x1 = -INFINITY;
         }
         const uint64_t p2 = tg::f2_pack(tg::ex2_approx(x0), tg::ex2_approx(x1));
-        const uint64_t d2 = tg::f2_add(tg::f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])), nd[c]);
+        const uint64_t d2 = tg::f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1]));  // dP - Delta
         const uint64_t dl2 = tg::f2_mul(p2, d2);
         cs2 = tg::f2_add(cs2, dl2);
         ta2 = tg::f2_fma(dl2, s2, ta2);
