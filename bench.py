@@ -56,8 +56,8 @@ NOMINAL_BF16_TFLOPS = 2250.0
 # at S = 8704, from one ncu capture of the kernel (its summary is kept with the
 # profiles).  It is reported only while the kernel sources are the ones that capture
 # measured.
-ATTENTION_TRAFFIC = {"sources_sha1": "825e579b131667fcffc0d9f146bc7abf44485e05",
-                     "read": 72824832, "write": 10231808}
+ATTENTION_TRAFFIC = {"sources_sha1": "d0c1fe096e48f54362f073462bcaa26f7d08a5f7",
+                     "read": 71617024, "write": 9345280}
 
 
 def attention_sources_sha1() -> str:

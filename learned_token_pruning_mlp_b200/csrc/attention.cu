@@ -22,8 +22,8 @@
 //     the first 64 columns of S_t and fed to the PV product straight from TMEM.
 //   * The key bias rides on the tensor core: with c_j = gain_h*log2(e)*s_j / scale
 //     (scale = tau*log2(e)/sqrt(D)), one extra K=16 MMA step multiplies a constant
-//     [1, 1, 0...] block of Q by a [hi(c_j), lo(c_j), 0...] block of K (c_j split
-//     into two bf16 parts, exact to 2^-16 relative), so S'_ij = q_i.k_j + c_j and the
+//     [1, 1, 1, 0...] block of Q by a [c0, c1, c2, 0...] block of K (c_j split into
+//     three bf16 parts, exact to 2^-24 relative), so S'_ij = q_i.k_j + c_j and the
 //     base-2 logit is scale * S'_ij: the softmax needs one FMA per logit, as without
 //     a bias.  tau < 0 negates the A operand (so the largest logit is still the
 //     largest S'); tau = 0 skips the Q.K steps.
@@ -126,8 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sQ = smem;                                  // [2][tile]
   uint8_t *sK = sQ + 2 * C::kTileBytes;                // [NS][tile]
   uint8_t *sV = sK + NS * C::kTileBytes;               // [NS][tile]
-  uint8_t *sQx = sV + NS * C::kTileBytes;              // [128 x 16] block of ones (columns 0, 1)
-  uint8_t *sKx = sQx + kExtBytes;                      // [NS][128 x 16] blocks of c_j (columns 0, 1)
+  uint8_t *sQx = sV + NS * C::kTileBytes;              // [128 x 16] block of ones (columns 0..2)
+  uint8_t *sKx = sQx + kExtBytes;                      // [NS][128 x 16] blocks of c_j (columns 0..2)
   AttnCtl *ctl = reinterpret_cast<AttnCtl *>(sKx + NS * kExtBytes);
   tg::pdl_wait();
   tg::pdl_trigger();
@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // constant [1, 1] columns of the extended Q block, zeros elsewhere (also in the c_j blocks)
   for (uint32_t w = threadIdx.x; w < (1 + NS) * kExtBytes / 4; w += kThreads) {
     uint32_t v = 0;
-    if (w < kExtLBO / 4 && (w & 3u) == 0) v = 0x3F803F80u;  // bf16 1.0 twice at the start of each row
+    if (w < kExtLBO / 4 && (w & 3u) == 0) v = 0x3F803F80u;  // bf16 1.0 in columns 0, 1 of each row
+    if (w < kExtLBO / 4 && (w & 3u) == 1) v = 0x00003F80u;  // and in column 2
     reinterpret_cast<uint32_t *>(sQx)[w] = v;
   }
   tg::fence_proxy_async_smem();
@@ -249,10 +250,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = e * 32 + lane;
         const int64_t kv = static_cast<int64_t>(j) * kBN + r;
         const float c = has_bias && kv < len ? cmul * key_scores[seg_start + kv] : 0.f;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(c);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(c - __bfloat162float(hi));
-        const __nv_bfloat162 pr = __halves2bfloat162(hi, lo);
-        *reinterpret_cast<__nv_bfloat162 *>(sKx + s * kExtBytes + r * 16) = pr;  // row r, columns 0..1
+        // c_j in three bf16 parts (their sum is c_j to 2^-24 relative)
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(c);
+        const float r1 = c - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+        uint8_t *row = sKx + s * kExtBytes + r * 16;  // row r, columns 0..2
+        *reinterpret_cast<__nv_bfloat162 *>(row) = __halves2bfloat162(p0, p1);
+        *reinterpret_cast<__nv_bfloat16 *>(row + 4) = p2;
       }
       tg::fence_proxy_async_smem();
       tg::mbar_arrive(tg::smem_addr(&ctl->bias_full[s]));

@@ -23,8 +23,8 @@
 //     once PV(t) has completed.
 //   * The key bias rides on the tensor core as in the two-tile kernel: with
 //     c_j = gain_h*log2(e)*s_j / scale (scale = tau*log2(e)/sqrt(D)), one extra K=16 MMA
-//     step multiplies a constant [1, 1, 0...] block by a [hi(c_j), lo(c_j), 0...] block
-//     (c_j split into two bf16 parts), so S'_ij = q_i.k_j + c_j and the base-2 logit is
+//     step multiplies a constant [1, 1, 1, 0...] block by a [c0, c1, c2, 0...] block
+//     (c_j split into three bf16 parts), so S'_ij = q_i.k_j + c_j and the base-2 logit is
 //     scale * S'_ij.  tau < 0 negates the A operand; tau = 0 skips the Q.K steps.
 //   * warp 0 (one lane) streams the K tiles and warp 2 (one lane, after allocating TMEM)
 //     the V tiles by TMA (128-byte swizzle); K and V stages are freed apart.  Warp 3 writes
@@ -200,8 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sStage = smem;                              // [tile] staged output tile
   uint8_t *sK = sStage + C::kTileBytes;                // [NS][tile]
   uint8_t *sV = sK + NS * C::kTileBytes;               // [NS][tile]
-  uint8_t *sQx = sV + NS * C::kTileBytes;              // [128 x 16] block of ones (columns 0, 1)
-  uint8_t *sKx = sQx + kExtBytes;                      // [NS][128 x 16] blocks of c_j (columns 0, 1)
+  uint8_t *sQx = sV + NS * C::kTileBytes;              // [128 x 16] block of ones (columns 0..2)
+  uint8_t *sKx = sQx + kExtBytes;                      // [NS][128 x 16] blocks of c_j (columns 0..2)
   float *sL = reinterpret_cast<float *>(sKx + NS * kExtBytes);  // [2 items][2 halves][128] partial row sums
   float *sM = sL + 4 * kBM;                                      // [2][128] row maxima (base-2 logit units)
   float *sXm = sM + 2 * kBM;                                     // [2 steps][2 halves][128] partial tile maxima
@@ -223,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // constant [1, 1] columns of the extended Q block, zeros elsewhere (also in the c_j blocks)
   for (uint32_t w = threadIdx.x; w < (1 + NS) * kExtBytes / 4; w += kThreads) {
     uint32_t v = 0;
-    if (w < kExtLBO / 4 && (w & 3u) == 0) v = 0x3F803F80u;  // bf16 1.0 twice at the start of each row
+    if (w < kExtLBO / 4 && (w & 3u) == 0) v = 0x3F803F80u;  // bf16 1.0 in columns 0, 1 of each row
+    if (w < kExtLBO / 4 && (w & 3u) == 1) v = 0x00003F80u;  // and in column 2
     reinterpret_cast<uint32_t *>(sQx)[w] = v;
   }
   tg::fence_proxy_async_smem();
@@ -333,10 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = e * 32 + lane;
             const int64_t kv = static_cast<int64_t>(j) * kBN + r;
             const float c = has_bias && kv < it.len ? cmul * key_scores[it.seg_start + kv] : 0.f;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(c);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(c - __bfloat162float(hi));
-            const __nv_bfloat162 pr = __halves2bfloat162(hi, lo);
-            *reinterpret_cast<__nv_bfloat162 *>(sKx + st * kExtBytes + r * 16) = pr;  // row r, columns 0..1
+            // c_j in three bf16 parts (their sum is c_j to 2^-24 relative)
+            const __nv_bfloat16 p0 = __float2bfloat16_rn(c);
+            const float r1 = c - __bfloat162float(p0);
+            const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+            uint8_t *row = sKx + st * kExtBytes + r * 16;  // row r, columns 0..2
+            *reinterpret_cast<__nv_bfloat162 *>(row) = __halves2bfloat162(p0, p1);
+            *reinterpret_cast<__nv_bfloat16 *>(row + 4) = p2;
           }
           tg::fence_proxy_async_smem();
           __syncwarp();

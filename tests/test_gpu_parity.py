@@ -60,7 +60,7 @@ def assert_gate_close(got, ref):
 
 # Relative weight error budget of the kernel: each probability is rounded to bf16 for the
 # PV product (2^-9 relative) and its logit carries fp32 rounding (the key bias split into
-# two bf16 parts is exact to 2^-18 of its size; below 2^-11 relative in every test here);
+# three bf16 parts is exact to 2^-24 of its size; below 2^-11 relative in every test here);
 # normalising by the sum of the same rounded weights at most doubles the effect, so the
 # output moves by at most (2^-8 + 2^-10) times the spread of the visible V rows.
 P_BUDGET = 2.0 ** -8 + 2.0 ** -10
