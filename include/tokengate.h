@@ -245,6 +245,11 @@ tg_status tg_gather(const tg_bf16 *hidden, int64_t n, int32_t d, const int32_t *
  * costs are measured against.
  * Sizes: S >= 0; D in {64, 128}; Hq a positive multiple of Hkv; S * Hq < 2^31.
  * Q, Kc, V and O 16-byte aligned.
+ * Two kernels serve this call and its varlen / training forms: one with two 128-row
+ * query tiles per CTA, and, when that grid (one CTA per 256 query rows, head and
+ * request, counted from max_seqlen) would hold at most 1.5 CTAs per SM, a persistent
+ * one that works through single query tiles.  Both are deterministic and held to the
+ * same tolerance; their outputs are not bitwise equal to each other.
  * -------------------------------------------------------------------------- */
 tg_status tg_gated_attention(const tg_bf16 *Q, const tg_bf16 *Kc, const tg_bf16 *V,
                              const float *s, const float *gain, float tau,
