@@ -3,8 +3,9 @@
 Each case draws its shapes and parameters from a fixed seed (so a failure reproduces):
 attention on both kernels (random length, heads, head dimension, temperature sign and
 size, gain and score scales, with or without scores), packed batches with random request
-lengths (empty ones included) and slack in max_seqlen, and the selector with random
-budgets, masks and tie-heavy scores.
+lengths (empty ones included) and slack in max_seqlen, the selector with random
+budgets, masks and tie-heavy scores, the backward (fed the oracle's forward) and the gate
+at random shapes.
 """
 import numpy as np
 import pytest
@@ -110,3 +111,44 @@ def test_topk_random_cases(seed):
     assert int(n_kept.item()) == len(ref)
     assert np.array_equal(kept[:len(ref)].cpu().numpy(), ref)
     assert tg.tg_get_device_error() & ~tg.TG_DEVERR_K_GT_NDOC == 0
+
+
+@pytest.mark.parametrize("seed", range(400, 416))
+def test_backward_random_cases(seed):
+    """The backward fed the oracle's forward (kernel parity) at random shapes, temperatures
+    (either sign), gains and score scales."""
+    from test_gpu_backward import _gpu_backward_on_oracle_forward, assert_kernel_close
+    rng = np.random.default_rng(seed)
+    S = int(rng.integers(64, 900))
+    Hkv = int(rng.choice([1, 2, 4]))
+    Hq = Hkv * int(rng.choice([1, 2, 4]))
+    D = int(rng.choice([64, 128]))
+    tau = float(rng.choice([-1.0, 1.0]) * rng.uniform(0.2, 2.5))
+    g = torch.Generator().manual_seed(seed)
+    Q = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    K = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    dO = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    s = torch.randn(S, generator=g) * float(rng.uniform(0.2, 3.0))
+    gain = 0.25 + torch.rand(Hq, generator=g) * float(rng.uniform(0.5, 1.5))
+    got = _gpu_backward_on_oracle_forward(Q, K, V, dO, s, gain, tau)
+    assert_kernel_close(got, oracle.gated_attention_backward(Q, K, V, s, gain, tau, dO))
+    assert tg.tg_get_device_error() == 0
+
+
+@pytest.mark.parametrize("seed", range(500, 510))
+def test_gate_random_cases(seed):
+    from test_gpu_parity import assert_gate_close
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 5000))
+    d = 8 * int(rng.integers(1, 300))
+    h = 16 * int(rng.integers(1, 17))
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(n, d, generator=g).to(torch.bfloat16)
+    W1 = (torch.randn(h, d, generator=g) / d ** 0.5).to(torch.bfloat16)
+    b1 = (torch.randn(h, generator=g) / d ** 0.5).to(torch.bfloat16)
+    W2 = (torch.randn(h, generator=g) / h ** 0.5).to(torch.bfloat16)
+    b2 = (torch.randn(1, generator=g) / h ** 0.5).to(torch.bfloat16)
+    got = tg.tg_gate_score(*(t.to(DEV) for t in (x, W1, b1, W2, b2)))
+    assert_gate_close(got.cpu().numpy(), oracle.gate_score(x, W1, b1, W2, b2))
+    assert tg.tg_get_device_error() == 0
